@@ -1,0 +1,431 @@
+"""Gated-prefill benchmark: one step = gate score + top-K + compaction + gated
+attention for one synthetic prompt batch, through libtokengate's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen_16k]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun, one process per GPU)
+are weak-scaling replicas: every rank processes its own prompt batch (its own
+seed), no data moves between GPUs, and the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "qwen_16k"
+L2_FLUSH_BYTES = 256 << 20
+METRIC = "gated-prefill input tok/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period_s=0.002):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nv = None
+        self._t = threading.Thread(target=self._loop, daemon=True)
+
+    def _loop(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def _dist_init(n_gpus):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        if world != n_gpus:
+            raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist.get_rank(), world, local
+    return 0, 1, 0
+
+
+def _max_over_ranks(x, world):
+    import torch
+    import torch.distributed as dist
+
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def _traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, or None once the kernel's
+    source has changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel, {}).get(workload)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "learned_token_pruning_gate_b200", "csrc", rec["source"])
+    if not os.path.exists(src) or _sha(src) != rec["sha256"]:
+        return None
+    return rec["bytes_per_launch"]
+
+
+def _sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def run_gpu(args):
+    import torch
+
+    import learned_token_pruning_gate_b200 as tg
+    from learned_token_pruning_gate_b200 import inputs as gen
+    from learned_token_pruning_gate_b200.pipeline import GatedLayer
+
+    rank, world, local = _dist_init(args.gpus)
+    torch.cuda.set_device(local)
+    base = gen.WORKLOADS[args.workload]
+    # weak scaling: rank r draws its own prompt batch (same shapes, seed + r)
+    w = gen.Workload(**{**base.__dict__, "seed": base.seed + 1000 * rank})
+    inp = gen.make_inputs(w)
+    dev = torch.device("cuda", local)
+    d = lambda t: t.to(dev).contiguous()  # noqa: E731
+    layer = GatedLayer(d(inp.h), d(inp.q), d(inp.k), d(inp.v), d(inp.W1), d(inp.b1), d(inp.w2),
+                       inp.b2, d(inp.gain), d(inp.temp), inp.cu_seqlens, inp.doc_begin,
+                       inp.doc_end, inp.budget, rope_theta=w.rope_theta, algo=tg.ALGO_AUTO)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    graph = layer.capture()
+
+    # ---- device-timed steps (inputs resident in HBM), CUDA graph replay --------
+    t_warm = time.time()
+    for i in range(max(args.warmup, 3)):
+        flush.zero_()
+        graph.replay()
+    while time.time() - t_warm < 0.3:  # let the clocks settle before timing
+        flush.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    _barrier(world)
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            flush.zero_()  # L2 flush outside the timed interval
+            ev[i][0].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    _barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = _max_over_ranks(float(np.sum(step_ms)), world)
+    if tg.device_status() != 0:
+        raise SystemExit("a kernel reported a timed-out wait")
+
+    # ---- per-kernel times for the roofline (same launches, one event pair each) --
+    n_k = min(K, 50)
+    kev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_k)] for s in GatedLayer.STAGES}
+    import ctypes
+
+    st = ctypes.c_void_p(stream.cuda_stream)
+    for i in range(n_k):
+        flush.zero_()
+        for s in GatedLayer.STAGES:
+            kev[s][i][0].record(stream)
+            getattr(layer, s)(st)
+            kev[s][i][1].record(stream)
+    torch.cuda.synchronize()
+    stage_ms = {s: float(np.mean([a.elapsed_time(b) for a, b in kev[s]])) for s in kev}
+
+    # ---- end to end: pinned host inputs -> device -> 4 C-ABI calls -> host -----
+    pinned = {n: getattr(inp, n).pin_memory() for n in ("h", "q", "k", "v")}
+    out_host = torch.empty(layer.out.shape, dtype=layer.out.dtype, pin_memory=True)
+    kept_host = torch.empty(layer.kept_idx.shape, dtype=torch.int32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_host.numel() * out_host.element_size() + kept_host.numel() * 4
+    n_e2e = max(min(K, 20), 3)
+
+    def e2e_step():
+        layer.h.copy_(pinned["h"], non_blocking=True)
+        layer.q.copy_(pinned["q"], non_blocking=True)
+        layer.k.copy_(pinned["k"], non_blocking=True)
+        layer.v.copy_(pinned["v"], non_blocking=True)
+        layer.run(stream.cuda_stream)
+        out_host.copy_(layer.out, non_blocking=True)
+        kept_host.copy_(layer.kept_idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
+    _barrier(world)
+
+    # ---- report -------------------------------------------------------------------
+    tokens = w.total_tokens
+    value = world * tokens * K / (total_ms / 1e3)
+    work = layer.work()
+    pk = _peaks()
+    us = {s: stage_ms[s] * 1e3 for s in stage_ms}
+    stages = {
+        "gate": {"us": us["gate"], "tflops": work["gate_flops"] / us["gate"] / 1e6,
+                 "gbs": work["gate_bytes"] / us["gate"] / 1e3},
+        "topk": {"us": us["topk"], "gbs": work["topk_bytes"] / us["topk"] / 1e3},
+        "gather": {"us": us["gather"], "gbs": work["gather_bytes"] / us["gather"] / 1e3},
+        "attention": {"us": us["attention"],
+                      "tflops": work["attn_flops"] / us["attention"] / 1e6},
+    }
+    for s in stages.values():
+        if "tflops" in s:
+            s["frac_tensor"] = s["tflops"] / pk["bf16"]
+        if "gbs" in s:
+            s["frac_hbm"] = s["gbs"] / pk["hbm"]
+    tg_us = us["topk"] + us["gather"]
+    stages["topk+gather"] = {"us": tg_us,
+                             "gbs": (work["topk_bytes"] + work["gather_bytes"]) / tg_us / 1e3}
+    stages["topk+gather"]["frac_hbm"] = stages["topk+gather"]["gbs"] / pk["hbm"]
+    dominant = max(("gate", "topk", "gather", "attention"), key=lambda s: us[s])
+    if dominant == "attention":
+        roof = {"kernel": "attn_tc_kernel", "bound": "tensor",
+                "achieved": stages["attention"]["tflops"], "peak": pk["bf16"], "unit": "TFLOP/s"}
+    elif dominant == "gate":
+        t_flop = work["gate_flops"] / (pk["bf16"] * 1e12)
+        t_byte = work["gate_bytes"] / (pk["hbm"] * 1e9)
+        if t_flop >= t_byte:
+            roof = {"kernel": "gate_tc_kernel", "bound": "tensor",
+                    "achieved": stages["gate"]["tflops"], "peak": pk["bf16"], "unit": "TFLOP/s"}
+        else:
+            roof = {"kernel": "gate_tc_kernel", "bound": "hbm", "achieved": stages["gate"]["gbs"],
+                    "peak": pk["hbm"], "unit": "GB/s"}
+    else:
+        roof = {"kernel": f"{dominant}_kernel", "bound": "hbm",
+                "achieved": stages[dominant]["gbs"], "peak": pk["hbm"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = _traffic(roof["kernel"], args.workload)
+    roof["peak_source"] = f"{pk['source']} (burst)"
+    e2e_value = world * tokens * n_e2e / (e2e_ms / 1e3)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "prompts_per_gpu": w.batch,
+                   "seq_len": list(w.seqlens), "question": list(w.question),
+                   "budget_K": list(w.budgets), "kept_M": w.kept_lengths(),
+                   "d_model": w.d_model, "gate": f"{w.d_model}->{w.d_hidden}->1",
+                   "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv x {w.head_dim}",
+                   "parallelism": f"replicas x{world} (independent prompts, no collective)",
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                   "timing": "CUDA events per step around a CUDA-graph replay of the 4 launches"},
+        "gpu_launches": 4 * K,
+        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": n_e2e},
+        "roofline": roof,
+        "stages": stages,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(inp, seconds=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def cpu_baseline(inp, seconds=15.0, repeats=1):
+    """The oracle, as it stands, on the host cores over a bounded sample of the
+    workload, extrapolated to the whole step by the work it does."""
+    import oracle
+
+    w = inp.w
+    N = w.total_tokens
+    rng = np.random.default_rng(0)
+    h32, W1 = inp.f32("h"), inp.f32("W1")
+    t_gate_row = None
+    n_rows = 256
+    while True:  # size the gate sample to ~1/3 of the budget
+        rows = rng.integers(0, N, n_rows)
+        t0 = time.perf_counter()
+        oracle.gate_score(h32, W1, inp.b1.numpy(), inp.w2.numpy(), inp.b2, rows=rows)
+        dt = time.perf_counter() - t0
+        t_gate_row = dt / n_rows
+        if dt > seconds / 3 or n_rows >= N:
+            break
+        n_rows = min(N, int(n_rows * max(2.0, (seconds / 3) / max(dt, 1e-3))))
+    gate_rows = n_rows
+    # top-K and compaction run whole on scores drawn for the sample
+    z = np.random.default_rng(1).standard_normal(N).astype(np.float32)  # score-shaped input
+    t0 = time.perf_counter()
+    kept, cu_kept = oracle.topk_select(z, inp.cu_seqlens, inp.doc_begin, inp.doc_end, inp.budget)
+    t_topk = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    qc = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("q"), w.n_q_heads, w.head_dim,
+                            w.rope_theta)
+    kc = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("k"), w.n_kv_heads, w.head_dim,
+                            w.rope_theta)
+    vc = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("v"))
+    hc = oracle.gather_rows(kept, inp.cu_seqlens, h32)
+    ls = oracle.logsig(kept, inp.cu_seqlens, inp.doc_begin, inp.doc_end, z)
+    t_gather = time.perf_counter() - t0
+    del hc
+    # attention: a sample of query rows, extrapolated by visible-key count
+    M = len(kept)
+    lens = np.diff(cu_kept)
+    vis_total = float(np.sum(lens * (lens + 1) / 2.0))
+    n_q = 32
+    while True:
+        rows = np.sort(rng.integers(0, M, n_q))
+        b_of = np.searchsorted(cu_kept, rows, side="right") - 1
+        vis = float(np.sum(rows - cu_kept[b_of] + 1))
+        t0 = time.perf_counter()
+        oracle.gated_attention(qc, kc, vc, cu_kept, ls, inp.gain.numpy(), inp.temp.numpy(),
+                               rows=rows)
+        dt = time.perf_counter() - t0
+        if dt > seconds / 3 or n_q >= M:
+            break
+        n_q = min(M, int(n_q * max(2.0, (seconds / 3) / max(dt, 1e-3))))
+    t_attn = dt * vis_total / max(vis, 1.0)
+    total = t_gate_row * N + t_topk + t_gather + t_attn
+    return {"value": N / total, "unit": "tok/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"gate on {gate_rows} of {N} tokens, top-K and compaction whole, "
+                       f"attention on {n_q} of {M} query rows (all heads); extrapolated by "
+                       f"tokens and by visible keys"),
+            "seconds_per_step_extrapolated": total}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle on this workload, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from learned_token_pruning_gate_b200 import inputs as gen
+
+    w = gen.WORKLOADS[args.workload]
+    inp = gen.make_inputs(w)
+    per_step = max(2.0, min(20.0, 120.0 / max(args.steps + args.warmup, 1)))
+    for _ in range(args.warmup):
+        cpu_baseline(inp, seconds=per_step / 4)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(inp, seconds=per_step))
+    wall = time.perf_counter() - t0
+    value = float(np.median([v["value"] for v in vals]))
+    cb = dict(vals[-1])
+    cb["value"] = value
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.total_tokens / value * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "seq_len": list(w.seqlens),
+                                        "budget_K": list(w.budgets)},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": wall, "oracle_threads": oracle.num_threads()}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

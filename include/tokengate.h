@@ -1,0 +1,199 @@
+/*
+ * tokengate.h -- C ABI of libtokengate.so, the B200 (sm_100a) gated-prefill hot
+ * path of TokenGate ("Adapting LLMs for Fast and Memory-Efficient Prefill with
+ * Learned Token Pruning").
+ *
+ * The method (abstract page; news write-ups, "how it works"): below a gate layer
+ * L every token is processed; at layer L a small MLP scores each token from its
+ * post-attention residual, a top-K selector keeps the highest-scoring document
+ * tokens while the question is never pruned, and the layers above L process only
+ * the kept tokens -- no KV entry exists for a dropped token.  To make the
+ * selection trainable, each kept token's score enters the attention logits above
+ * the gate as a bias (the Mixture-of-Experts router trick) with a per-head
+ * learned gain, and a per-head learned temperature corrects for each query
+ * seeing fewer keys.  The four calls below are that forward pass, one call per
+ * step:
+ *
+ *     tg_gate_score -> tg_topk_select -> tg_compact_gather -> tg_gated_attention
+ *
+ * Conventions shared by every call
+ *   - Device pointers point to memory on the current CUDA device; "host" arrays
+ *     are ordinary host memory read synchronously during the call.
+ *   - The caller owns and allocates every buffer.  The library allocates no
+ *     device memory, keeps no state between calls and never synchronises the
+ *     stream: each call validates its arguments, enqueues kernels on `stream`
+ *     and returns.
+ *   - A prompt batch is packed row-major ("varlen"): prompt b owns rows
+ *     [cu_seqlens[b], cu_seqlens[b+1]) of every per-token tensor.  Each prompt
+ *     is [document | question] in any arrangement: doc_begin/doc_end give the
+ *     prunable document span relative to the prompt's first row (the `{state}`
+ *     span of the reference prompt template); every token outside it is
+ *     protected (always kept).  At most TG_MAX_BATCH prompts per call.
+ *   - Errors: a call that returns anything but TG_OK has enqueued no work.
+ *     TG_ERR_CUDA means a launch failed; tg_last_error_message() describes the
+ *     most recent error on the calling host thread.
+ *   - Kept rows: with n_doc = doc_end - doc_begin and K = budget, prompt b keeps
+ *     M_b = min(K, n_doc) + (N_b - n_doc) rows, in ascending original order.
+ */
+#ifndef TOKENGATE_H_
+#define TOKENGATE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TG_API __attribute__((visibility("default")))
+#else
+#define TG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tg_stream_t; /* same type as cudaStream_t; NULL = legacy default */
+
+typedef enum {
+    TG_OK = 0,
+    TG_ERR_INVALID_ARG = 1,  /* null pointer, negative size or budget, bad span */
+    TG_ERR_SHAPE = 2,        /* inconsistent sizes between arguments */
+    TG_ERR_DTYPE = 3,        /* unknown tg_dtype */
+    TG_ERR_ALIGNMENT = 4,    /* a pointer or row pitch is not 16-byte aligned */
+    TG_ERR_UNSUPPORTED = 5,  /* valid but outside what the kernels implement */
+    TG_ERR_CUDA = 6,         /* a CUDA runtime/driver call or launch failed */
+    TG_ERR_DEVICE_CHECK = 7  /* a kernel reported a failure (see tg_device_status) */
+} tg_status;
+
+typedef enum { TG_BF16 = 0, TG_FP32 = 1 } tg_dtype;
+
+/* Kernel selection for the two contraction steps. */
+typedef enum {
+    TG_ALGO_AUTO = 0,    /* tensor-core kernel when the shape allows it, else CUDA cores */
+    TG_ALGO_SIMT = 1,    /* CUDA-core (FFMA) kernel; every dtype and shape it accepts */
+    TG_ALGO_TCGEN05 = 2  /* tcgen05/TMEM tensor-core kernel; TG_ERR_UNSUPPORTED if the shape
+                            or dtype does not allow it (bf16 only) */
+} tg_algo;
+
+#define TG_MAX_BATCH 128
+
+/* Human-readable name of a status code (static string). */
+TG_API const char* tg_status_string(tg_status status);
+
+/* Description of the most recent failed call on this host thread (static buffer). */
+TG_API const char* tg_last_error_message(void);
+
+/* Library version string, e.g. "0.1.0 sm_100a". */
+TG_API const char* tg_version(void);
+
+/*
+ * Device-side status word: kernels never trap; a bounded wait that gives up
+ * (a pipeline barrier that did not complete within ~2 s) sets a bit here and
+ * the kernel exits early with its outputs undefined.  Synchronises `stream`,
+ * writes the accumulated bits to *bits_out (0 = no failure) and clears them.
+ * Returns TG_ERR_DEVICE_CHECK when bits were set.
+ */
+TG_API tg_status tg_device_status(tg_stream_t stream, uint32_t* bits_out);
+
+/*
+ * Host-only helper: validates a prompt batch and writes the kept-row offsets
+ * cu_kept_h[0..batch] (cu_kept_h[b+1] - cu_kept_h[b] = M_b) so the caller can
+ * size the outputs of the later calls.  All arrays are host memory.
+ */
+TG_API tg_status tg_kept_offsets(int32_t batch, const int32_t* cu_seqlens_h, const int32_t* doc_begin_h,
+                          const int32_t* doc_end_h, const int32_t* budget_h, int32_t* cu_kept_h);
+
+/*
+ * Step 1 -- gate score (pages: "at layer L a small MLP scores each token from
+ * its post-attention residual").  For every token j:
+ *     z[j] = sum_u w2[u] * GELU(sum_c W1[u,c] h[j,c] + b1[u]) + b2
+ * with the exact (erf) GELU, products accumulated in fp32.
+ *   h        device [n_tokens, d_model], dtype, row-major, 16-byte aligned
+ *   W1       device [d_hidden, d_model], same dtype, row-major (K-major)
+ *   b1, w2   device [d_hidden] fp32;  b2 host scalar
+ *   z_out    device [n_tokens] fp32
+ *   algo     tg_algo.  The tcgen05 kernel needs bf16, d_model % 64 == 0 and
+ *            d_hidden a multiple of 32 in [32, 256].
+ */
+TG_API tg_status tg_gate_score(const void* h, tg_dtype dtype, int64_t n_tokens, int32_t d_model,
+                        const void* W1, const float* b1, int32_t d_hidden, const float* w2,
+                        float b2, float* z_out, int32_t algo, tg_stream_t stream);
+
+/*
+ * Step 2 -- top-K over each prompt's document span, question protected
+ * (pages: "a top-K selector keeps the highest-scoring tokens"; "only the
+ * document part of the prompt is pruned, the question is never touched"; the
+ * user budget is max_kept_prefill_tokens).  Selection order: larger fp32 score
+ * first; +0.0 and -0.0 are equal; equal scores by lower index; NaN after every
+ * number.  Exactly min(K, n_doc) document tokens are kept, so the result is
+ * unique.
+ *   z             device [total_tokens] fp32 scores
+ *   batch, cu_seqlens_h[batch+1], doc_begin_h/doc_end_h/budget_h[batch]: host
+ *   kept_idx_out  device [M] int32 global row ids, ascending within a prompt,
+ *                 prompts in order (M = sum M_b, see tg_kept_offsets)
+ *   cu_kept_out   device [batch+1] int32 kept-row offsets (may be NULL)
+ * Limits: N_b <= 360448 tokens per prompt (TG_ERR_UNSUPPORTED beyond).
+ */
+TG_API tg_status tg_topk_select(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                         const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                         const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
+                         tg_stream_t stream);
+
+/* One tensor to compact: rows of `row_elems` elements, pitch = row_elems. */
+typedef struct {
+    const void* src;     /* device [total_tokens, row_elems] */
+    void* dst;           /* device [M, row_elems] */
+    int32_t row_elems;   /* elements per row; row bytes must be a multiple of 16 */
+    int32_t rope_heads;  /* 0 = plain copy; else the first rope_heads*head_dim elements
+                            are rope_heads heads rotated by RoPE (rotate-half pairing,
+                            angle pos * theta^(-2i/head_dim), pos = original position
+                            within the prompt, angles evaluated in fp64) */
+} tg_gather_tensor;
+
+#define TG_MAX_GATHER_TENSORS 8
+
+/*
+ * Step 3 -- compaction (pages: "layers above L process only the kept K tokens
+ * and create no KV cache for the removed ones").  For each kept row i:
+ *     dst_t[i] = src_t[kept_idx[i]]            (RoPE applied where requested)
+ *     logsig_out[i] = log sigmoid(z[kept_idx[i]]) for document tokens, 0 for
+ *                     question tokens (the per-key bias term of step 4)
+ *   kept_idx      device [m_total] from tg_topk_select
+ *   prompt arrays host, as for tg_topk_select (m_total must equal sum M_b)
+ *   tensors       host array of n_tensors (<= TG_MAX_GATHER_TENSORS) entries
+ *   head_dim      RoPE head size (even, <= 256) when any rope_heads > 0
+ *   z             device [total_tokens] fp32 (may be NULL when logsig_out is NULL)
+ *   logsig_out    device [m_total] fp32 or NULL
+ */
+TG_API tg_status tg_compact_gather(const int32_t* kept_idx, int64_t m_total, int32_t batch,
+                            const int32_t* cu_seqlens_h, const int32_t* doc_begin_h,
+                            const int32_t* doc_end_h, const int32_t* budget_h, tg_dtype dtype,
+                            const tg_gather_tensor* tensors, int32_t n_tensors, int32_t head_dim,
+                            double rope_theta, const float* z, float* logsig_out,
+                            tg_stream_t stream);
+
+/*
+ * Step 4 -- token-gated causal GQA attention over the kept rows (pages: the
+ * kept tokens' scores become a bias on the attention logits above the gate,
+ * scaled by a per-head learned gain; a per-head learned temperature corrects
+ * for each query seeing fewer keys).  For prompt b, query row i, head h:
+ *     logit_j = (q_i . k_j) / (sqrt(head_dim) * temp[h]) + gain[h] * logsig[j]
+ *     out_i   = sum_{j <= i in prompt b} softmax_j(logit) v_j
+ *     lse[h, i] = log sum_j exp(logit_j)            (natural log)
+ * with kv head = h / (n_q_heads / n_kv_heads).  logsig == NULL means no bias.
+ *   q    device [M, n_q_heads, head_dim];  k, v device [M, n_kv_heads, head_dim]
+ *   cu_kept_h  host [batch+1] kept-row offsets (M = cu_kept_h[batch])
+ *   gain, temp device [n_q_heads] fp32 (temp > 0)
+ *   out  device [M, n_q_heads, head_dim], dtype;  lse device [n_q_heads, M] or NULL
+ *   algo tg_algo; the tcgen05 kernel needs bf16 and head_dim in {64, 128}.
+ */
+TG_API tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dtype dtype,
+                             int32_t batch, const int32_t* cu_kept_h, int32_t n_q_heads,
+                             int32_t n_kv_heads, int32_t head_dim, const float* logsig,
+                             const float* gain, const float* temp, void* out, float* lse,
+                             int32_t algo, tg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_H_ */

@@ -1,1 +1,256 @@
-"""TokenGate gated-prefill hot path for B200 (sm_100a)."""
+"""TokenGate gated-prefill hot path for B200 (sm_100a).
+
+Thin Python binding over ``libtokengate.so`` (C ABI in ``include/tokengate.h``).
+This module only marshals arguments: torch tensors supply device memory and the
+current CUDA stream, every step runs in the library's kernels.  There is no
+fallback: if the library is missing or a call fails, an exception is raised.
+
+The four calls follow the method's forward pass (TokenGate abstract page;
+news write-ups, "how it works"):
+
+    gate_score -> topk_select -> compact_gather -> gated_attention
+
+``gated_prefill`` chains them for one prompt batch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+__all__ = [
+    "TG_BF16", "TG_FP32", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "TokenGateError",
+    "library", "kept_offsets", "gate_score", "topk_select", "compact_gather", "gated_attention",
+    "gated_prefill", "device_status", "EXPORTED_SYMBOLS",
+]
+
+TG_BF16, TG_FP32 = 0, 1
+ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
+MAX_BATCH = 128
+MAX_GATHER_TENSORS = 8
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtokengate.so")
+
+EXPORTED_SYMBOLS = (
+    "tg_status_string", "tg_last_error_message", "tg_version", "tg_device_status",
+    "tg_kept_offsets", "tg_gate_score", "tg_topk_select", "tg_compact_gather",
+    "tg_gated_attention",
+)
+
+
+class TokenGateError(RuntimeError):
+    """A libtokengate call returned an error status."""
+
+    def __init__(self, fn, status, message):
+        super().__init__(f"{fn}: {status}: {message}")
+        self.status = status
+
+
+class GatherTensor(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p),
+                ("row_elems", ctypes.c_int32), ("rope_heads", ctypes.c_int32)]
+
+
+_lib = None
+_vp, _i32, _i64, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+_i32p = ctypes.POINTER(ctypes.c_int32)
+
+
+def library():
+    """Load libtokengate.so (built by ``python -m learned_token_pruning_gate_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m learned_token_pruning_gate_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.tg_status_string.restype = ctypes.c_char_p
+    L.tg_status_string.argtypes = [ctypes.c_int]
+    L.tg_last_error_message.restype = ctypes.c_char_p
+    L.tg_version.restype = ctypes.c_char_p
+    L.tg_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.tg_kept_offsets.argtypes = [_i32, _i32p, _i32p, _i32p, _i32p, _i32p]
+    L.tg_gate_score.argtypes = [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, _i32, _vp, _f32, _vp,
+                                _i32, _vp]
+    L.tg_topk_select.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp]
+    L.tg_compact_gather.argtypes = [_vp, _i64, _i32, _i32p, _i32p, _i32p, _i32p, ctypes.c_int,
+                                    ctypes.POINTER(GatherTensor), _i32, _i32, ctypes.c_double,
+                                    _vp, _vp, _vp]
+    L.tg_gated_attention.argtypes = [_vp, _vp, _vp, ctypes.c_int, _i32, _i32p, _i32, _i32, _i32,
+                                     _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+    for name in EXPORTED_SYMBOLS:
+        if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
+            getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(fn, status):
+    if status != 0:
+        L = library()
+        raise TokenGateError(fn, L.tg_status_string(status).decode(),
+                             L.tg_last_error_message().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _host_i32(a):
+    arr = np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+    return arr, arr.ctypes.data_as(_i32p)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return TG_BF16
+    if t.dtype == torch.float32:
+        return TG_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libtokengate operates on CUDA tensors only")
+
+
+def device_status(stream=None):
+    """Synchronise and return (and clear) the device status bits (0 = no failure)."""
+    bits = ctypes.c_uint32(0)
+    st = stream if stream is not None else _stream()
+    rc = library().tg_device_status(st, ctypes.byref(bits))
+    if rc not in (0, 7):
+        _check("tg_device_status", rc)
+    return bits.value
+
+
+def kept_offsets(cu_seqlens, doc_begin, doc_end, budget) -> np.ndarray:
+    """Host-side kept-row offsets cu_kept [B+1] (validates the prompt batch)."""
+    cu, cu_p = _host_i32(cu_seqlens)
+    s, s_p = _host_i32(doc_begin)
+    e, e_p = _host_i32(doc_end)
+    k, k_p = _host_i32(budget)
+    out = np.zeros(len(s) + 1, np.int32)
+    _check("tg_kept_offsets", library().tg_kept_offsets(len(s), cu_p, s_p, e_p, k_p,
+                                                        out.ctypes.data_as(_i32p)))
+    return out
+
+
+def gate_score(h, W1, b1, w2, b2, out=None, algo=ALGO_AUTO):
+    """z = w2 . GELU(W1 h + b1) + b2 for every row of h [n, d]."""
+    _need_cuda(h, W1, b1, w2)
+    n, d = h.shape
+    dg = W1.shape[0]
+    if W1.shape[1] != d or W1.dtype != h.dtype:
+        raise ValueError("W1 must be [d_hidden, d_model] with h's dtype")
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=h.device)
+    _check("tg_gate_score", library().tg_gate_score(
+        _ptr(h), _dtype_code(h), n, d, _ptr(W1), _ptr(b1), dg, _ptr(w2), float(b2), _ptr(out),
+        algo, _stream(h.device)))
+    return out
+
+
+def topk_select(z, cu_seqlens, doc_begin, doc_end, budget, kept_idx=None, cu_kept=None):
+    """Per-prompt top-K of the document span (question kept).
+
+    Returns (kept_idx [M] int32 device, cu_kept [B+1] int32 device, cu_kept_host).
+    """
+    _need_cuda(z)
+    cu, cu_p = _host_i32(cu_seqlens)
+    s, s_p = _host_i32(doc_begin)
+    e, e_p = _host_i32(doc_end)
+    k, k_p = _host_i32(budget)
+    host = kept_offsets(cu, s, e, k)
+    M = int(host[-1])
+    if kept_idx is None:
+        kept_idx = torch.empty(max(M, 1), dtype=torch.int32, device=z.device)[:M]
+    if cu_kept is None:
+        cu_kept = torch.empty(len(s) + 1, dtype=torch.int32, device=z.device)
+    _check("tg_topk_select", library().tg_topk_select(
+        _ptr(z), len(s), cu_p, s_p, e_p, k_p, _ptr(kept_idx), _ptr(cu_kept), _stream(z.device)))
+    return kept_idx, cu_kept, host
+
+
+def compact_gather(kept_idx, cu_seqlens, doc_begin, doc_end, budget, tensors, rope_heads=None,
+                   head_dim=0, rope_theta=1e6, z=None, logsig_out=None, outs=None):
+    """Gather kept rows of each tensor in ``tensors`` (RoPE where rope_heads[i] > 0).
+
+    Returns (list of compacted tensors, logsig [M] fp32 or None).
+    """
+    if len(tensors) > MAX_GATHER_TENSORS:
+        raise ValueError("too many tensors")
+    _need_cuda(kept_idx, z, *tensors)
+    cu, cu_p = _host_i32(cu_seqlens)
+    s, s_p = _host_i32(doc_begin)
+    e, e_p = _host_i32(doc_end)
+    k, k_p = _host_i32(budget)
+    M = kept_idx.shape[0]
+    dtypes = {t.dtype for t in tensors}
+    if len(dtypes) > 1:
+        raise ValueError("all gathered tensors must share one dtype")
+    dcode = _dtype_code(tensors[0]) if tensors else TG_BF16
+    rope_heads = rope_heads or [0] * len(tensors)
+    if outs is None:
+        outs = [torch.empty((M,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+                for t in tensors]
+    arr = (GatherTensor * max(len(tensors), 1))()
+    for i, (src, dst) in enumerate(zip(tensors, outs)):
+        if not src.is_contiguous() or not dst.is_contiguous():
+            raise ValueError("gather tensors must be contiguous")
+        arr[i].src = src.data_ptr()
+        arr[i].dst = dst.data_ptr()
+        arr[i].row_elems = src[0].numel() if src.shape[0] > 0 else int(np.prod(src.shape[1:]))
+        arr[i].rope_heads = int(rope_heads[i])
+    if z is not None and logsig_out is None:
+        logsig_out = torch.empty(M, dtype=torch.float32, device=z.device)
+    dev = (tensors[0].device if tensors else z.device)
+    _check("tg_compact_gather", library().tg_compact_gather(
+        _ptr(kept_idx), M, len(s), cu_p, s_p, e_p, k_p, dcode, arr, len(tensors), head_dim,
+        float(rope_theta), _ptr(z), _ptr(logsig_out), _stream(dev)))
+    return outs, logsig_out
+
+
+def gated_attention(q, k, v, cu_kept_host, logsig=None, gain=None, temp=None, out=None,
+                    lse=None, algo=ALGO_AUTO, want_lse=False):
+    """Token-gated causal GQA attention over packed kept rows.
+
+    q [M, Hq, d], k/v [M, Hkv, d]; cu_kept_host [B+1] host offsets.
+    Returns (out [M, Hq, d], lse [Hq, M] or None).
+    """
+    _need_cuda(q, k, v, logsig, gain, temp)
+    M, Hq, dh = q.shape
+    Hkv = k.shape[1]
+    cu, cu_p = _host_i32(cu_kept_host)
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((Hq, M), dtype=torch.float32, device=q.device)
+    _check("tg_gated_attention", library().tg_gated_attention(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), len(cu) - 1, cu_p, Hq, Hkv, dh, _ptr(logsig),
+        _ptr(gain), _ptr(temp), _ptr(out), _ptr(lse), algo, _stream(q.device)))
+    return out, lse
+
+
+def gated_prefill(h, q, k, v, W1, b1, w2, b2, gain, temp, cu_seqlens, doc_begin, doc_end,
+                  budget, rope_theta=1e6, algo=ALGO_AUTO, want_lse=False):
+    """One gated layer: score, select, compact, attend.  Returns a dict of device tensors."""
+    z = gate_score(h, W1, b1, w2, b2, algo=algo)
+    kept_idx, cu_kept, cu_kept_host = topk_select(z, cu_seqlens, doc_begin, doc_end, budget)
+    Hq, dh = q.shape[1], q.shape[2]
+    (h_c, q_c, k_c, v_c), logsig = compact_gather(
+        kept_idx, cu_seqlens, doc_begin, doc_end, budget, [h, q, k, v],
+        rope_heads=[0, Hq, k.shape[1], 0], head_dim=dh, rope_theta=rope_theta, z=z)
+    o, lse = gated_attention(q_c, k_c, v_c, cu_kept_host, logsig, gain, temp, algo=algo,
+                             want_lse=want_lse)
+    return dict(z=z, kept_idx=kept_idx, cu_kept=cu_kept, cu_kept_host=cu_kept_host, h=h_c, q=q_c,
+                k=k_c, v=v_c, logsig=logsig, out=o, lse=lse)

@@ -1,0 +1,159 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and rejects invalid arguments with the documented status
+before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import learned_token_pruning_gate_b200 as tg
+from learned_token_pruning_gate_b200 import build as tgbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tokengate.h")
+
+OK, INVALID, SHAPE, DTYPE, ALIGN, UNSUP, CUDA = 0, 1, 2, 3, 4, 5, 6
+FAKE = ctypes.c_void_p(0x10000)      # aligned, never dereferenced by a rejected call
+FAKE_ODD = ctypes.c_void_p(0x10008)  # 8-byte aligned only
+
+
+@pytest.fixture(scope="module")
+def L():
+    tgbuild.build()
+    return tg.library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tg_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared_functions()
+    assert declared, "no declarations parsed"
+    assert set(declared) == set(tg.EXPORTED_SYMBOLS)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_only_abi_symbols_are_exported(L):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", tg.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert {s for s in syms if s.startswith("tg_")} == set(tg.EXPORTED_SYMBOLS)
+
+
+def test_status_strings_and_version(L):
+    assert L.tg_status_string(0) == b"TG_OK"
+    assert L.tg_status_string(5) == b"TG_ERR_UNSUPPORTED"
+    assert b"sm_100a" in L.tg_version()
+
+
+def _arr(a):
+    a = np.ascontiguousarray(a, np.int32)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def test_kept_offsets_matches_definition(L):
+    cu, cu_p = _arr([0, 100, 100, 350])
+    s, s_p = _arr([10, 0, 0])
+    e, e_p = _arr([90, 0, 250])
+    k, k_p = _arr([30, 5, 1000])
+    out = np.zeros(4, np.int32)
+    rc = L.tg_kept_offsets(3, cu_p, s_p, e_p, k_p, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    assert rc == OK
+    # M_b = min(K, n_doc) + (N_b - n_doc)
+    assert out.tolist() == [0, 30 + 20, 50 + 0, 50 + 250]
+
+
+@pytest.mark.parametrize("cu,s,e,k,code", [
+    ([0, 10], [0], [11], [1], INVALID),   # span past the end
+    ([0, 10], [5], [4], [1], INVALID),    # reversed span
+    ([0, 10], [0], [5], [-1], INVALID),   # negative budget
+    ([1, 10], [0], [5], [1], INVALID),    # cu_seqlens[0] != 0
+    ([0, 10, 5], [0, 0], [5, 0], [1, 1], INVALID),  # decreasing offsets
+])
+def test_prompt_validation(L, cu, s, e, k, code):
+    _, cu_p = _arr(cu)
+    _, s_p = _arr(s)
+    _, e_p = _arr(e)
+    _, k_p = _arr(k)
+    out = np.zeros(len(s) + 1, np.int32)
+    assert L.tg_kept_offsets(len(s), cu_p, s_p, e_p, k_p,
+                             out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))) == code
+    assert L.tg_topk_select(FAKE, len(s), cu_p, s_p, e_p, k_p, FAKE, FAKE, None) == code
+    assert b"" != L.tg_last_error_message()
+
+
+def test_topk_limits(L):
+    B = 129
+    _, cu_p = _arr(np.arange(B + 1) * 4)
+    _, s_p = _arr(np.zeros(B))
+    _, e_p = _arr(np.full(B, 2))
+    _, k_p = _arr(np.ones(B))
+    assert L.tg_topk_select(FAKE, B, cu_p, s_p, e_p, k_p, FAKE, FAKE, None) == UNSUP
+    _, cu_p = _arr([0, 400000])
+    _, s_p = _arr([0])
+    _, e_p = _arr([399000])
+    _, k_p = _arr([10])
+    assert L.tg_topk_select(FAKE, 1, cu_p, s_p, e_p, k_p, FAKE, FAKE, None) == UNSUP
+
+
+def test_gate_validation(L):
+    g = L.tg_gate_score
+    assert g(FAKE, 7, 16, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 0, None) == DTYPE
+    assert g(FAKE, 0, -1, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 0, None) == INVALID
+    assert g(FAKE_ODD, 0, 16, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 0, None) == ALIGN
+    assert g(FAKE, 0, 16, 60, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 0, None) == ALIGN  # 120-byte rows
+    assert g(FAKE, 1, 16, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 2, None) == UNSUP  # tcgen05 + fp32
+    assert g(FAKE, 0, 16, 96, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 2, None) == UNSUP  # d % 64
+    assert g(FAKE, 0, 16, 64, FAKE, FAKE, 48, FAKE, 0.0, FAKE, 2, None) == UNSUP  # dg % 32
+    assert g(FAKE, 0, 16, 64, FAKE, FAKE, 512, FAKE, 0.0, FAKE, 2, None) == UNSUP  # dg > 256
+    assert g(FAKE, 0, 16, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 9, None) == INVALID
+    assert g(None, 0, 16, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 0, None) == INVALID
+    assert g(None, 0, 0, 64, None, None, 32, None, 0.0, None, 0, None) == OK  # empty: no-op
+
+
+def test_gather_validation(L):
+    _, cu_p = _arr([0, 10])
+    _, s_p = _arr([0])
+    _, e_p = _arr([8])
+    _, k_p = _arr([4])
+    t = (tg.GatherTensor * 1)()
+    t[0].src, t[0].dst, t[0].row_elems, t[0].rope_heads = 0x10000, 0x20000, 64, 1
+    f = L.tg_compact_gather
+    assert f(FAKE, 5, 1, cu_p, s_p, e_p, k_p, 0, t, 1, 64, 1e6, FAKE, FAKE, None) == SHAPE  # M=6
+    assert f(FAKE, 6, 1, cu_p, s_p, e_p, k_p, 0, t, 1, 96, 1e6, FAKE, FAKE, None) == SHAPE  # 96>64
+    assert f(FAKE, 6, 1, cu_p, s_p, e_p, k_p, 0, t, 1, 40, 1e6, FAKE, FAKE, None) == UNSUP
+    assert f(FAKE, 6, 1, cu_p, s_p, e_p, k_p, 0, t, 1, 64, 0.5, FAKE, FAKE, None) == INVALID
+    t[0].row_elems = 60  # 120-byte rows
+    t[0].rope_heads = 0
+    assert f(FAKE, 6, 1, cu_p, s_p, e_p, k_p, 0, t, 1, 0, 1e6, FAKE, FAKE, None) == ALIGN
+    assert f(FAKE, 6, 1, cu_p, s_p, e_p, k_p, 0, t, 9, 0, 1e6, FAKE, FAKE, None) == INVALID
+
+
+def test_attention_validation(L):
+    _, ck = _arr([0, 100])
+    a = L.tg_gated_attention
+    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 6, 128, None, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
+    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 8, 96, None, FAKE, FAKE, FAKE, None, 0, None) == UNSUP
+    assert a(FAKE, FAKE, FAKE, 1, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, 2, None) == UNSUP
+    assert a(FAKE_ODD, FAKE, FAKE, 0, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, 0,
+             None) == ALIGN
+    _, bad = _arr([0, 100, 50])
+    assert a(FAKE, FAKE, FAKE, 0, 2, bad, 16, 8, 128, None, FAKE, FAKE, FAKE, None, 0,
+             None) == INVALID
+
+
+def test_no_gpu_means_cuda_error_not_crash(L):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    bits = ctypes.c_uint32(0)
+    assert L.tg_device_status(None, ctypes.byref(bits)) == CUDA

@@ -1,0 +1,131 @@
+"""GPU parity: gate score (tcgen05 and CUDA-core kernels) and top-K selection,
+through the C ABI, against the fp64 oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import learned_token_pruning_gate_b200 as tg
+from learned_token_pruning_gate_b200 import inputs as gen
+from tests.parity_utils import GATE_ATOL, assert_close, dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    tg.library()
+    yield
+    assert tg.device_status() == 0, "a kernel reported a timed-out wait"
+
+
+# ---- gate ------------------------------------------------------------------
+
+def _rand_gate(n, d, dg, dtype, seed, needle=False):
+    rng = np.random.Generator(np.random.Philox(seed))
+    h = rng.standard_normal((n, d), dtype=np.float32)
+    W1 = rng.standard_normal((dg, d), dtype=np.float32) * 0.02
+    if needle:
+        h[n // 3] *= 6.0
+    b1 = rng.standard_normal(dg, dtype=np.float32) * 0.02
+    w2 = rng.standard_normal(dg, dtype=np.float32) * 0.02
+    t = torch.float32 if dtype == "fp32" else torch.bfloat16
+    return (torch.from_numpy(h).to(t), torch.from_numpy(W1).to(t), torch.from_numpy(b1),
+            torch.from_numpy(w2), 0.013)
+
+
+@pytest.mark.parametrize("n,d,dg,dtype,algo", [
+    (1024, 256, 64, "fp32", tg.ALGO_AUTO),       # the tiny fp32 layer
+    (1000, 2048, 256, "bf16", tg.ALGO_TCGEN05),  # Qwen-shaped, ragged last tile
+    (1000, 2048, 256, "bf16", tg.ALGO_SIMT),
+    (129, 128, 32, "bf16", tg.ALGO_TCGEN05),     # two tiles, one row in the second
+    (1, 64, 32, "bf16", tg.ALGO_TCGEN05),
+    (300, 320, 96, "bf16", tg.ALGO_TCGEN05),
+    (5000, 512, 224, "bf16", tg.ALGO_TCGEN05),   # more tiles than SMs reuse the TMEM ring
+    (77, 100, 20, "fp32", tg.ALGO_SIMT),
+])
+def test_gate_parity(oracle, n, d, dg, dtype, algo):
+    h, W1, b1, w2, b2 = _rand_gate(n, d, dg, dtype, seed=n * 7 + d, needle=True)
+    z = tg.gate_score(dev(h), dev(W1), dev(b1), dev(w2), b2, algo=algo)
+    ref = oracle.gate_score(h.float().numpy(), W1.float().numpy(), b1.numpy(), w2.numpy(), b2)
+    assert_close("z", z.cpu().numpy(), ref, GATE_ATOL, 0.0)
+    if dtype == "fp32":  # fp32 products: far inside the bar
+        assert_close("z(fp32)", z.cpu().numpy(), ref, 2e-5, 0.0)
+
+
+@pytest.mark.parametrize("name", ["qwen_16k", "qwen_128k", "ragged_4"])
+def test_gate_full_size_sampled(oracle, name):
+    w = gen.WORKLOADS[name]
+    inp = gen.make_inputs(w, with_qkv=False)
+    z = tg.gate_score(dev(inp.h), dev(inp.W1), dev(inp.b1), dev(inp.w2), inp.b2).cpu().numpy()
+    N = w.total_tokens
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([
+        rng.integers(0, N, 384), np.arange(N - 130, N), np.arange(0, 130),
+        np.concatenate(inp.needle_rows)[:64]]))
+    ref = oracle.gate_score(inp.f32("h"), inp.f32("W1"), inp.b1.numpy(), inp.w2.numpy(), inp.b2,
+                            rows=rows)
+    assert_close("z", z[rows], ref, GATE_ATOL, 0.0)
+    assert np.isfinite(z).all()
+
+
+# ---- top-K -------------------------------------------------------------------
+
+def _topk_both(oracle, z, cu, s, e, k):
+    kept, cu_kept, host = tg.topk_select(torch.from_numpy(z).cuda(), cu, s, e, k)
+    ref_kept, ref_cu = oracle.topk_select(z, cu, s, e, k)
+    np.testing.assert_array_equal(host, ref_cu)
+    np.testing.assert_array_equal(cu_kept.cpu().numpy(), ref_cu)
+    np.testing.assert_array_equal(kept.cpu().numpy(), ref_kept)
+
+
+@pytest.mark.parametrize("n", [1, 2, 31, 100, 1000, 4097, 16384, 131072])
+@pytest.mark.parametrize("kfrac", [0.0, 0.001, 0.25, 0.999, 1.0, 2.0])
+def test_topk_bit_exact_single(oracle, n, kfrac):
+    z = gen.random_scores(n, seed=n)
+    q = min(256, n // 4)
+    n_doc = n - q
+    K = int(round(kfrac * n_doc))
+    _topk_both(oracle, z, [0, n], [0], [n_doc], [K])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_bit_exact_varlen(oracle, seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 12))
+    lens = rng.integers(0, 20000, size=B)
+    lens[rng.random(B) < 0.2] = 0
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    s = np.array([rng.integers(0, L + 1) for L in lens], np.int32)
+    e = np.array([rng.integers(ss, L + 1) for ss, L in zip(s, lens)], np.int32)
+    k = np.array([rng.integers(0, max(ee - ss, 1) + 3) for ss, ee in zip(s, e)], np.int32)
+    z = gen.random_scores(int(cu[-1]), seed=100 + seed)
+    _topk_both(oracle, z, cu, s, e, k)
+
+
+def test_topk_ties_everywhere(oracle):
+    n = 50000
+    z = np.full(n, 0.5, np.float32)
+    z[::7] = 0.25
+    z[::1000] = np.nan
+    z[5::9] = -0.0
+    z[6::9] = 0.0
+    for K in (1, 6000, 30000, 49000):
+        _topk_both(oracle, z, [0, n], [100], [n - 100], [K])
+
+
+def test_topk_question_in_the_middle_and_front(oracle):
+    z = gen.random_scores(30000, seed=3)
+    cu = [0, 10000, 30000]
+    _topk_both(oracle, z, cu, [500, 0], [9000, 19000], [700, 12345])
+
+
+@pytest.mark.parametrize("name,seed", [("qwen_128k", 3), ("ragged_4", 4), ("qwen_32k_k1024", 2),
+                                       ("qwen_32k_k4096", 2), ("qwen_32k_k8192", 2)])
+def test_topk_full_size(oracle, name, seed):
+    w = gen.WORKLOADS[name]
+    cu = np.concatenate([[0], np.cumsum(w.seqlens)]).astype(np.int32)
+    e = np.array([n - q for n, q in zip(w.seqlens, w.question)], np.int32)
+    z = gen.random_scores(int(cu[-1]), seed=seed, specials=False)
+    _topk_both(oracle, z, cu, np.zeros(w.batch, np.int32), e, np.array(w.budgets, np.int32))
