@@ -110,27 +110,6 @@ def _dist_init(n_gpus):
     return 0, 1, 0
 
 
-def _max_over_ranks(x, world):
-    import torch
-    import torch.distributed as dist
-
-    if world == 1:
-        return float(x)
-    t = torch.tensor([float(x)], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def _barrier(world):
-    import torch
-    import torch.distributed as dist
-
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-
-
 def _traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu capture, or None once the kernel's
     source has changed since the capture."""
@@ -155,13 +134,13 @@ def run_gpu(args):
 
     import learned_token_pruning_gate_b200 as tg
     from learned_token_pruning_gate_b200 import inputs as gen
+    from learned_token_pruning_gate_b200 import dist as tgd
     from learned_token_pruning_gate_b200.pipeline import GatedLayer
 
     rank, world, local = _dist_init(args.gpus)
     torch.cuda.set_device(local)
-    base = gen.WORKLOADS[args.workload]
-    # weak scaling: rank r draws its own prompt batch (same shapes, seed + r)
-    w = gen.Workload(**{**base.__dict__, "seed": base.seed + 1000 * rank})
+    # weak scaling: rank r draws its own prompt batch (same shapes, its own seed)
+    w = tgd.rank_workload(gen.WORKLOADS[args.workload], rank)
     inp = gen.make_inputs(w)
     dev = torch.device("cuda", local)
     d = lambda t: t.to(dev).contiguous()  # noqa: E731
@@ -184,7 +163,7 @@ def run_gpu(args):
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
-    _barrier(world)
+    tgd.barrier()
     with ClockSampler(local) as clocks:
         for i in range(K):
             flush.zero_()  # L2 flush outside the timed interval
@@ -192,9 +171,9 @@ def run_gpu(args):
             graph.replay()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-    _barrier(world)
+    tgd.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = _max_over_ranks(float(np.sum(step_ms)), world)
+    total_ms = tgd.max_over_ranks(float(np.sum(step_ms)), device=dev)
     if tg.device_status() != 0:
         raise SystemExit("a kernel reported a timed-out wait")
 
@@ -233,19 +212,19 @@ def run_gpu(args):
 
     for _ in range(3):
         e2e_step()
-    _barrier(world)
+    tgd.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(n_e2e):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
-    _barrier(world)
+    e2e_ms = tgd.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    tgd.barrier()
 
     # ---- report -------------------------------------------------------------------
     tokens = w.total_tokens
-    value = world * tokens * K / (total_ms / 1e3)
+    value = tgd.aggregate_throughput(tokens, K, total_ms, world)
     work = layer.work()
     pk = _peaks()
     us = {s: stage_ms[s] * 1e3 for s in stage_ms}
@@ -285,7 +264,7 @@ def run_gpu(args):
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = _traffic(roof["kernel"], args.workload)
     roof["peak_source"] = f"{pk['source']} (burst)"
-    e2e_value = world * tokens * n_e2e / (e2e_ms / 1e3)
+    e2e_value = tgd.aggregate_throughput(tokens, n_e2e, e2e_ms, world)
 
     result = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": K,
@@ -411,6 +390,29 @@ def run_reference(args):
         "wall_s": wall, "oracle_threads": oracle.num_threads()}), flush=True)
 
 
+def run_ncu_case(args):
+    """Untimed: build the workload and run `--steps` plain steps (for ncu captures)."""
+    import torch
+
+    import learned_token_pruning_gate_b200 as tg
+    from learned_token_pruning_gate_b200 import inputs as gen
+    from learned_token_pruning_gate_b200.pipeline import GatedLayer
+
+    w = gen.WORKLOADS[args.workload]
+    inp = gen.make_inputs(w)
+    d = lambda t: t.cuda().contiguous()  # noqa: E731
+    layer = GatedLayer(d(inp.h), d(inp.q), d(inp.k), d(inp.v), d(inp.W1), d(inp.b1), d(inp.w2),
+                       inp.b2, d(inp.gain), d(inp.temp), inp.cu_seqlens, inp.doc_begin,
+                       inp.doc_end, inp.budget, rope_theta=w.rope_theta)
+    for _ in range(args.steps):
+        layer.run()
+    torch.cuda.synchronize()
+    if tg.device_status() != 0:
+        raise SystemExit("a kernel reported a timed-out wait")
+    print(json.dumps({"ncu_case": args.workload, "steps": args.steps, "N": layer.N,
+                      "M": layer.M}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -420,8 +422,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="untimed: run --steps plain steps of the workload (profiling)")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.ncu_case:
+        run_ncu_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
