@@ -1,0 +1,562 @@
+// Token-gated causal GQA attention, tensor-core path (bf16, head_dim 64/128).
+//
+// TokenGate adds each kept key's gate score to the attention logits above the
+// gate as a bias scaled by a per-head learned gain (the Mixture-of-Experts
+// router trick) and divides q.k by a per-head learned temperature:
+//     logit_ij = q_i.k_j / (sqrt(d) tau_h) + g_h l_j,     j <= i in the prompt.
+// In the log2 domain t = s * log2e/(sqrt(d) tau_h) + g_h log2e l_j, so bias
+// and temperature cost one FMA per logit.
+//
+// Work item = (prompt, 128-query tile, pair of query heads sharing one KV
+// head).  Both heads of a pair need exactly the same K/V tiles (0..tile), so a
+// K/V tile is loaded once and feeds two independent softmax warpgroups that
+// take turns with the tensor core (while one computes softmax, the tensor core
+// runs the other's P.V and next Q.K^T).  The kernel is persistent: one CTA per
+// SM walks the items in order of decreasing length (longest first), so the
+// causal imbalance is spread across SMs.
+//
+//   warp 0     TMA: both Q tiles of an item, then K and V tiles (128 keys)
+//              into a ring of shared-memory stages (128-byte swizzle)
+//   warp 1     TMEM owner (512 columns: S_a, S_b, O_a, O_b) and the single
+//              tcgen05.mma issuer: S_x = Q_x K^T, O_x += P_x V with P_x read
+//              from TMEM (bf16 written over S_x) and V MN-major from smem.
+//              Issue order S_a0 S_b0 | PV_a0 S_a1 | PV_b0 S_b1 | ... relies on
+//              tcgen05.mma executing in issue order.
+//   warps 2-3  idle (they only complete warpgroup 0 for the register split)
+//   warps 4-7  softmax for head a, warps 8-11 for head b: one query row per
+//              thread; packed fp32x2 math; causal mask on the diagonal tile;
+//              lazy rescaling: O is rescaled in TMEM only when a row's max
+//              grows by more than 2^8 (the P.V of the previous tile is known
+//              complete then, because this tile's S commit tracks it).
+//              Epilogue: O / l -> bf16 -> global, LSE.
+#include "tg_internal.cuh"
+
+namespace tg {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kThreads = 384;  // 3 warpgroups
+// Register split (launch: 384 threads x 168 = 64512): warpgroup 0 (TMA, MMA and
+// two idle warps) shrinks to 104 per thread, the two softmax warpgroups grow to
+// 192: 128*104 + 256*192 = 62464 <= 64512.
+constexpr int kRegsProducer = 104;
+constexpr int kRegsSoftmax = 192;
+static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * 168, "register split");
+constexpr int kBM = 128;       // queries per tile
+constexpr int kBN = 128;       // keys per tile
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct TcParams {
+  int32_t kept_start[kMaxBatch + 1];
+  int32_t order[kMaxBatch];      // prompts by query-tile count, descending
+  int32_t nt_sorted[kMaxBatch];  // their query-tile counts
+  const float* logsig;
+  const float* gain;
+  const float* temp;
+  __nv_bfloat16* out;
+  float* lse;
+  uint32_t* status;
+  int32_t batch;
+  int32_t m_total;
+  int32_t hq;
+  int32_t group;          // query heads per KV head
+  int32_t pairs_per_kvh;  // ceil(group / 2)
+  int32_t pairs;          // head pairs per (prompt, query tile) = hkv * pairs_per_kvh
+  int32_t n_items;
+};
+
+template <int DH>
+struct Lay {
+  static constexpr uint32_t kChunks = DH / 64;
+  static constexpr uint32_t kBox = 128 * 128;           // 128 rows x 64 bf16 (16 KB)
+  static constexpr uint32_t kTile = kChunks * kBox;     // one 128-row Q/K/V tile
+  static constexpr int kStages = DH == 64 ? 4 : 2;
+  static constexpr uint32_t kQa = 0;
+  static constexpr uint32_t kQb = kTile;
+  static constexpr uint32_t kK = 2 * kTile;
+  static constexpr uint32_t kV = kK + kStages * kTile;
+  static constexpr uint32_t kBias = kV + kStages * kTile;  // [2 heads][2 parity][128] fp32
+  static constexpr uint32_t kBars = kBias + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kMisc = kBars + 32 * 8;
+  static constexpr uint32_t kTotal = kMisc + 16;
+  static constexpr uint32_t kDynSmem = kTotal + 1024;
+};
+
+// barrier slots
+enum {
+  kQFull = 0,
+  kQEmpty = 1,
+  kSFull = 2,   // [2]
+  kPFull = 4,   // [2]
+  kOFull = 6,   // [2]
+  kOFree = 8,   // [2]
+  kKFull = 10,  // [stages]
+};
+
+struct Item {
+  int b, t, ha, hb, hk;
+  bool has_b;
+};
+
+// Number of items at query-tile levels >= t.
+__device__ __forceinline__ int items_at_or_above(const TcParams& p, int t) {
+  int s = 0;
+  for (int k = 0; k < p.batch; ++k) {
+    const int d = p.nt_sorted[k] - t;
+    if (d <= 0) break;
+    s += d;
+  }
+  return s * p.pairs;
+}
+
+// Item of rank r in longest-first order: levels (query tile index) descending,
+// then prompts (longest first), then head pairs.
+__device__ __forceinline__ Item decode_item(const TcParams& p, int r) {
+  int lo = 0, hi = p.nt_sorted[0] - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (items_at_or_above(p, mid) > r) lo = mid; else hi = mid - 1;
+  }
+  const int idx = r - items_at_or_above(p, lo + 1);
+  const int k = idx / p.pairs, pr = idx - k * p.pairs;
+  Item it;
+  it.b = p.order[k];
+  it.t = lo;
+  const int g = pr / p.pairs_per_kvh, pp = pr - g * p.pairs_per_kvh;
+  it.hk = g;
+  it.ha = g * p.group + 2 * pp;
+  it.hb = it.ha + 1;
+  it.has_b = 2 * pp + 1 < p.group;
+  return it;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ TcParams p) {
+  using L = Lay<DH>;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  float* s_bias = reinterpret_cast<float*>(smem + L::kBias);
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  auto k_full = [&](int s) { return bar(kKFull + s); };
+  auto v_full = [&](int s) { return bar(kKFull + S + s); };
+  auto kv_empty = [&](int s) { return bar(kKFull + 2 * S + s); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    mbar_init(bar(kQFull), 1);
+    mbar_init(bar(kQEmpty), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(kSFull + x), 1);
+      mbar_init(bar(kPFull + x), 128);
+      mbar_init(bar(kOFull + x), 1);
+      mbar_init(bar(kOFree + x), 128);
+    }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int rs = 0;
+      uint32_t rph = 0, q_waits = 0;
+      bool ok = true;
+      for (int r = blockIdx.x; ok && r < p.n_items; r += gridDim.x) {
+        const Item it = decode_item(p, r);
+        const int32_t kstart = p.kept_start[it.b];
+        if (!(ok = mbar_wait(bar(kQEmpty), (q_waits++ & 1) ^ 1, abort_flag, p.status,
+                             kDevTimeoutAttn)))
+          break;
+        mbar_arrive_expect_tx(bar(kQFull), L::kTile * (it.has_b ? 2 : 1));
+        for (uint32_t c = 0; c < L::kChunks; ++c) {
+          tma_load_2d(sb + L::kQa + c * L::kBox, &tm_q, it.ha * DH + c * 64, kstart + it.t * kBM,
+                      bar(kQFull));
+          if (it.has_b)
+            tma_load_2d(sb + L::kQb + c * L::kBox, &tm_q, it.hb * DH + c * 64,
+                        kstart + it.t * kBM, bar(kQFull));
+        }
+        for (int j = 0; j <= it.t; ++j) {
+          if (!(ok = mbar_wait(kv_empty(rs), rph ^ 1, abort_flag, p.status, kDevTimeoutAttn)))
+            break;
+          const int krow = kstart + j * kBN;
+          mbar_arrive_expect_tx(k_full(rs), L::kTile);
+          for (uint32_t c = 0; c < L::kChunks; ++c)
+            tma_load_2d(sb + L::kK + rs * L::kTile + c * L::kBox, &tm_k, it.hk * DH + c * 64, krow,
+                        k_full(rs));
+          mbar_arrive_expect_tx(v_full(rs), L::kTile);
+          for (uint32_t c = 0; c < L::kChunks; ++c)
+            tma_load_2d(sb + L::kV + rs * L::kTile + c * L::kBox, &tm_v, it.hk * DH + c * 64, krow,
+                        v_full(rs));
+          if (++rs == S) {
+            rs = 0;
+            rph ^= 1;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, DH, false, true);
+      auto wt = [&](uint32_t b, uint32_t par) {
+        return mbar_wait(b, par, abort_flag, p.status, kDevTimeoutAttn);
+      };
+      // S_x = Q_x K^T for head x with the K tile in stage s
+      auto issue_s = [&](int x, int s) {
+        const uint32_t qb = sb + (x ? L::kQb : L::kQa);
+        const uint32_t kb = sb + L::kK + s * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
+          umma_ss(tmem + x * 128, sw128_desc(qb + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
+                  idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(kSFull + x));
+      };
+      // O_x (+)= P_x V with the V tile in stage s
+      auto issue_pv = [&](int x, int s, bool acc) {
+        const uint32_t vb = sb + L::kV + s * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
+                  sw128_desc(vb + kk * 2048, L::kBox, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+      };
+      int rs = 0;
+      uint32_t rph = 0, q_waits = 0, p_waits[2] = {0, 0}, of_waits[2] = {0, 0};
+      bool ok = true;
+      for (int r = blockIdx.x; ok && r < p.n_items; r += gridDim.x) {
+        const Item it = decode_item(p, r);
+        const int n_kv = it.t + 1;
+        if (!(ok = wt(bar(kQFull), q_waits++ & 1))) break;
+        if (!(ok = wt(k_full(rs), rph))) break;
+        tc_fence_after();
+        issue_s(0, rs);
+        if (it.has_b) issue_s(1, rs);
+        if (n_kv == 1) umma_commit(bar(kQEmpty));
+        for (int j = 0; ok && j < n_kv; ++j) {
+          int ns = rs + 1;
+          uint32_t nph = rph;
+          if (ns == S) {
+            ns = 0;
+            nph ^= 1;
+          }
+          const bool more = j + 1 < n_kv;
+          // head a: P_a(j) V_j, then S_a(j+1)
+          if (!(ok = wt(bar(kPFull + 0), p_waits[0]++ & 1))) break;
+          if (j == 0 && !(ok = wt(bar(kOFree + 0), (of_waits[0]++ & 1) ^ 1))) break;
+          if (!(ok = wt(v_full(rs), rph))) break;
+          tc_fence_after();
+          issue_pv(0, rs, j > 0);
+          if (!more) umma_commit(bar(kOFull + 0));
+          if (more) {
+            if (!(ok = wt(k_full(ns), nph))) break;
+            tc_fence_after();
+            issue_s(0, ns);
+            if (!it.has_b && j + 2 == n_kv) umma_commit(bar(kQEmpty));
+          }
+          // head b: P_b(j) V_j, then S_b(j+1)
+          if (it.has_b) {
+            if (!(ok = wt(bar(kPFull + 1), p_waits[1]++ & 1))) break;
+            if (j == 0 && !(ok = wt(bar(kOFree + 1), (of_waits[1]++ & 1) ^ 1))) break;
+            tc_fence_after();
+            issue_pv(1, rs, j > 0);
+            if (!more) umma_commit(bar(kOFull + 1));
+          }
+          umma_commit(kv_empty(rs));  // V_j (and K_j) no longer needed once these finish
+          if (more && it.has_b) {
+            issue_s(1, ns);
+            if (j + 2 == n_kv) umma_commit(bar(kQEmpty));
+          }
+          rs = ns;
+          rph = nph;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- softmax warpgroups ----------------
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int x = (warp - 4) >> 2;  // 0: head a (warps 4-7), 1: head b (warps 8-11)
+    const int quarter = warp & 3;
+    const int rl = quarter * 32 + lane;  // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + x * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + x * 128;
+    uint32_t s_waits = 0, o_waits = 0, tile_ctr = 0;
+    bool ok = true;
+    for (int r = blockIdx.x; ok && r < p.n_items; r += gridDim.x) {
+      const Item it = decode_item(p, r);
+      if (x == 1 && !it.has_b) continue;
+      const int head = x ? it.hb : it.ha;
+      const int32_t kstart = p.kept_start[it.b];
+      const int32_t len = p.kept_start[it.b + 1] - kstart;
+      const int n_kv = it.t + 1;
+      const float scale = kLog2e / (sqrtf(static_cast<float>(DH)) * __ldg(p.temp + head));
+      const float gl = __ldg(p.gain + head) * kLog2e;
+      const float2 sc2 = make_float2(scale, scale);
+      float m = -INFINITY, l = 0.0f;
+      for (int j = 0; j < n_kv; ++j) {
+        float* bias = s_bias + (x * 2 + (tile_ctr & 1)) * 128;
+        ++tile_ctr;
+        {
+          const int key = j * kBN + rl;
+          bias[rl] = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
+        }
+        named_barrier(1 + x, 128);
+        if (!(ok = mbar_wait(bar(kSFull + x), s_waits++ & 1, abort_flag, p.status,
+                             kDevTimeoutAttn)))
+          break;
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+        // t = s * scale + bias; tile max
+        float mx = -INFINITY;
+        const float4* b4 = reinterpret_cast<const float4*>(bias);
+        if (j + 1 < n_kv) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 bb = b4[(c * 32 + e) >> 2];
+              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
+                                     sc2, make_float2(bb.x, bb.y));
+              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
+                                     sc2, make_float2(bb.z, bb.w));
+              sr[c][e] = __float_as_uint(t0.x);
+              sr[c][e + 1] = __float_as_uint(t0.y);
+              sr[c][e + 2] = __float_as_uint(t1.x);
+              sr[c][e + 3] = __float_as_uint(t1.y);
+              mx = max3f(mx, t0.x, t0.y);
+              mx = max3f(mx, t1.x, t1.y);
+            }
+          }
+        } else {  // diagonal tile: key column c is visible to row rl iff c <= rl
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const int col = c * 32 + e;
+              const float4 bb = b4[col >> 2];
+              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
+                                     sc2, make_float2(bb.x, bb.y));
+              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
+                                     sc2, make_float2(bb.z, bb.w));
+              if (col > rl) t0.x = -INFINITY;
+              if (col + 1 > rl) t0.y = -INFINITY;
+              if (col + 2 > rl) t1.x = -INFINITY;
+              if (col + 3 > rl) t1.y = -INFINITY;
+              sr[c][e] = __float_as_uint(t0.x);
+              sr[c][e + 1] = __float_as_uint(t0.y);
+              sr[c][e + 2] = __float_as_uint(t1.x);
+              sr[c][e + 3] = __float_as_uint(t1.y);
+              mx = max3f(mx, t0.x, t0.y);
+              mx = max3f(mx, t1.x, t1.y);
+            }
+          }
+        }
+        // lazy rescale: move the reference max only when it grows by > 2^8
+        float alpha = 1.0f;
+        const bool grow = mx > m + kRescaleLog2;
+        if (grow) {
+          alpha = exp2_approx(m - mx);
+          m = mx;
+        }
+        // The previous tile's P.V is complete (this tile's S commit tracked it), so
+        // O may be rescaled in place.  Warp-uniform: tcgen05.ld/st are collective.
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t orow[32];
+            tmem_ld32(t_o + c * 32, orow);
+            tmem_ld_wait(orow);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v2 = __fmul2_rn(
+                  make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
+                  make_float2(alpha, alpha));
+              orow[e] = __float_as_uint(v2.x);
+              orow[e + 1] = __float_as_uint(v2.y);
+            }
+            tmem_st32(t_o + c * 32, orow);
+          }
+        }
+        // p = 2^(t - m), row sum, and P (bf16 pairs) over the first 64 columns of S,
+        // 32 keys (16 columns) at a time
+        const float2 nm2 = make_float2(-m, -m);
+        float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 a2 = __fadd2_rn(
+                make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), nm2);
+            const float2 p2 = make_float2(exp2_approx(a2.x), exp2_approx(a2.y));
+            acc = __fadd2_rn(acc, p2);
+            __nv_bfloat162 pp = __floats2bfloat162_rn(p2.x, p2.y);
+            pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
+          }
+          tmem_st16(t_s + c * 16, pk);
+        }
+        l = fmaf(l, alpha, acc.x + acc.y);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(kPFull + x));
+      }
+      if (!ok) break;
+      // epilogue: O / l
+      if (!(ok = mbar_wait(bar(kOFull + x), o_waits++ & 1, abort_flag, p.status,
+                           kDevTimeoutAttn)))
+        break;
+      tc_fence_after();
+      const int qi = it.t * kBM + rl;
+      const float inv = 1.0f / l;
+      __nv_bfloat16* out = p.out + (static_cast<int64_t>(kstart + qi) * p.hq + head) * DH;
+#pragma unroll
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t orow[32];
+        tmem_ld32(t_o + c * 32, orow);
+        tmem_ld_wait(orow);
+        if (qi < len) {
+          uint32_t pkd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(orow[2 * e]) * inv,
+                                                      __uint_as_float(orow[2 * e + 1]) * inv);
+            pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kOFree + x));
+      if (p.lse && qi < len)
+        p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (m + log2f(l)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int DH>
+tg_status launch_dh(const void* q, const void* k, const void* v, TcParams& p, int hkv,
+                    cudaStream_t st) {
+  using Ly = Lay<DH>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t M = static_cast<uint64_t>(p.m_total);
+  if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(p.hq) * DH, M,
+                           static_cast<uint64_t>(p.hq) * DH * 2, 64, kBM) ||
+      !encode_tmap_2d_bf16(&tk, k, static_cast<uint64_t>(hkv) * DH, M,
+                           static_cast<uint64_t>(hkv) * DH * 2, 64, kBN) ||
+      !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(hkv) * DH, M,
+                           static_cast<uint64_t>(hkv) * DH * 2, 64, kBN))
+    return set_error(TG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q/k/v");
+  tg_status r = cuda_check(cudaFuncSetAttribute(attn_tc_kernel<DH>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(Ly::kDynSmem)),
+                           "attn smem attribute");
+  if (r != TG_OK) return r;
+  int grid = num_sms();
+  if (grid > p.n_items) grid = p.n_items;
+  attn_tc_kernel<DH><<<grid, kThreads, Ly::kDynSmem, st>>>(tq, tk, tv, p);
+  return cuda_check(cudaGetLastError(), "attn_tc launch");
+}
+
+}  // namespace
+
+tg_status launch_attn_tc(const void* q, const void* k, const void* v, const PromptTable& pt,
+                         int max_len, int hq, int hkv, int dh, const float* logsig,
+                         const float* gain, const float* temp, void* out, float* lse,
+                         cudaStream_t st) {
+  (void)max_len;
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  p.batch = pt.batch;
+  for (int b = 0; b <= pt.batch; ++b) p.kept_start[b] = pt.kept_start[b];
+  // prompts by query-tile count, descending (stable)
+  int nt[kMaxBatch];
+  for (int b = 0; b < pt.batch; ++b) {
+    nt[b] = (pt.kept_start[b + 1] - pt.kept_start[b] + kBM - 1) / kBM;
+    p.order[b] = b;
+  }
+  for (int i = 1; i < pt.batch; ++i) {
+    const int xb = p.order[i];
+    int j = i - 1;
+    while (j >= 0 && nt[p.order[j]] < nt[xb]) {
+      p.order[j + 1] = p.order[j];
+      --j;
+    }
+    p.order[j + 1] = xb;
+  }
+  int64_t tiles = 0;
+  for (int i = 0; i < pt.batch; ++i) {
+    p.nt_sorted[i] = nt[p.order[i]];
+    tiles += p.nt_sorted[i];
+  }
+  p.logsig = logsig;
+  p.gain = gain;
+  p.temp = temp;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.status = device_status_word();
+  if (!p.status) return set_error(TG_ERR_CUDA, "device status word unavailable");
+  p.m_total = pt.kept_start[pt.batch];
+  p.hq = hq;
+  p.group = hq / hkv;
+  p.pairs_per_kvh = (p.group + 1) / 2;
+  p.pairs = hkv * p.pairs_per_kvh;
+  const int64_t n_items = tiles * p.pairs;
+  if (n_items == 0) return TG_OK;
+  if (n_items > 0x7FFFFFFF) return set_error(TG_ERR_UNSUPPORTED, "too many attention tiles");
+  p.n_items = static_cast<int32_t>(n_items);
+  if (dh == 64) return launch_dh<64>(q, k, v, p, hkv, st);
+  return launch_dh<128>(q, k, v, p, hkv, st);
+}
+
+}  // namespace tg
