@@ -330,12 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float gl = __ldg(p.gain + head) * kLog2e;
       const float2 sc2 = make_float2(scale, scale);
       float m = -INFINITY, l = 0.0f;
+      // this thread's key of the next tile's bias, loaded one tile ahead
+      float next_bias = (p.logsig && rl < len) ? gl * __ldg(p.logsig + kstart + rl) : 0.0f;
       for (int j = 0; j < n_kv; ++j) {
         float* bias = s_bias + (x * 2 + (tile_ctr & 1)) * 128;
         ++tile_ctr;
-        {
-          const int key = j * kBN + rl;
-          bias[rl] = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
+        bias[rl] = next_bias;
+        if (j + 1 < n_kv) {
+          const int key = (j + 1) * kBN + rl;
+          next_bias = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
         }
         named_barrier(1 + x, 128);
         if (!(ok = mbar_wait(bar(kSFull + x), s_waits++ & 1, abort_flag, p.status,
@@ -348,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
         // t = s * scale + bias; tile max
-        float mx = -INFINITY;
+        // four independent max chains (short dependency chains for two warps per scheduler)
+        float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         const float4* b4 = reinterpret_cast<const float4*>(bias);
         if (j + 1 < n_kv) {
 #pragma unroll
@@ -364,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               sr[c][e + 1] = __float_as_uint(t0.y);
               sr[c][e + 2] = __float_as_uint(t1.x);
               sr[c][e + 3] = __float_as_uint(t1.y);
-              mx = max3f(mx, t0.x, t0.y);
-              mx = max3f(mx, t1.x, t1.y);
+              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
+              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
             }
           }
         } else {  // diagonal tile: key column c is visible to row rl iff c <= rl
@@ -387,11 +391,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               sr[c][e + 1] = __float_as_uint(t0.y);
               sr[c][e + 2] = __float_as_uint(t1.x);
               sr[c][e + 3] = __float_as_uint(t1.y);
-              mx = max3f(mx, t0.x, t0.y);
-              mx = max3f(mx, t1.x, t1.y);
+              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
+              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
             }
           }
         }
+        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
         // lazy rescale: move the reference max only when it grows by > 2^8
         float alpha = 1.0f;
         const bool grow = mx > m + kRescaleLog2;
@@ -421,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(t - m), row sum, and P (bf16 pairs) over the first 64 columns of S,
         // 32 keys (16 columns) at a time
         const float2 nm2 = make_float2(-m, -m);
-        float2 acc = make_float2(0.0f, 0.0f);
+        float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
@@ -430,13 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 a2 = __fadd2_rn(
                 make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), nm2);
             const float2 p2 = make_float2(exp2_approx(a2.x), exp2_approx(a2.y));
-            acc = __fadd2_rn(acc, p2);
+            acc[(e >> 1) & 1] = __fadd2_rn(acc[(e >> 1) & 1], p2);
             __nv_bfloat162 pp = __floats2bfloat162_rn(p2.x, p2.y);
             pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
           }
           tmem_st16(t_s + c * 16, pk);
         }
-        l = fmaf(l, alpha, acc.x + acc.y);
+        l = fmaf(l, alpha, (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(kPFull + x));

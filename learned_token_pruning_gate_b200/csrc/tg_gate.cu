@@ -228,6 +228,187 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---- tensor-core path on CTA pairs (tcgen05 cta_group::2) ---------------------
+// Same dataflow as gate_tc_kernel, but a cluster of two CTAs computes one
+// 256-row tile with M=256 MMAs: each CTA stages its own 128 residual rows and
+// only half of W1 (d_hidden/2 rows), so every SM streams 32 KB per k-block
+// instead of 48 KB and the W1 re-read from L2 per residual row halves.  The
+// even CTA issues the MMAs for both; its barriers count both CTAs' TMA bytes and
+// both epilogues' releases, and it signals the odd CTA's barriers with a second
+// commit.
+// A stage covers 128 columns of the residual (two adjacent 128-byte swizzle boxes
+// per row), so each row contributes 256 contiguous bytes per TMA round.
+constexpr int kStages2 = 3;
+constexpr int kBK2 = 128;
+
+struct Gate2Layout {
+  uint32_t stage_bytes, a_bytes, a_box, b_box;
+  uint32_t bars_off, misc_off, b1_off, w2_off, total;
+  __host__ __device__ Gate2Layout(int dg) {
+    a_box = kBM * kBK * 2;                             // 128 rows x 64 cols
+    b_box = static_cast<uint32_t>(dg / 2) * kBK * 2;   // dg/2 rows x 64 cols
+    a_bytes = 2 * a_box;
+    stage_bytes = a_bytes + 2 * b_box;
+    bars_off = kStages2 * stage_bytes;
+    misc_off = bars_off + 24 * 8;
+    b1_off = misc_off + 16;
+    w2_off = b1_off + 256 * 4;
+    total = w2_off + 256 * 4;
+  }
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gate_tc2_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ GateTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const Gate2Layout L(p.dg);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars_off);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc_off + 4);
+  float* s_b1 = reinterpret_cast<float*>(smem + L.b1_off);
+  float* s_w2 = reinterpret_cast<float*>(smem + L.w2_off);
+  // barrier indices: full[0..5], empty[6..11], tmem_full[12..13], tmem_empty[14..15]
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  auto leader_bar = [&](int i) { return mapa_shared(bar(i), 0); };
+  auto peer_bar = [&](int i) { return mapa_shared(bar(i), 1); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = p.d / kBK2;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(bar(s), 1);
+      mbar_init(bar(6 + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar(12 + a), 1);
+      mbar_init(bar(14 + a), 256);  // both CTAs' epilogue threads
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+    prefetch_tmap(&tm_h);
+    prefetch_tmap(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp >= 2) {
+    for (int i = threadIdx.x - 64; i < p.dg; i += 128) {
+      s_b1[i] = p.b1[i];
+      s_w2[i] = p.w2[i];
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers and TMEM of both CTAs are ready
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!(ok = mbar_wait(bar(6 + stage), phase ^ 1, abort_flag, p.status, kDevTimeoutGate)))
+            break;
+          const uint32_t sa = smem_u32(smem + stage * L.stage_bytes);
+          if (leader) mbar_arrive_expect_tx(bar(stage), 2 * L.stage_bytes);
+          for (int c = 0; c < 2; ++c)
+            tma_load_2d_pair(sa + c * L.a_box, &tm_h, kb * kBK2 + c * kBK,
+                             tile * 2 * kBM + rank * kBM, leader_bar(stage), pol_stream);
+          for (int c = 0; c < 2; ++c)
+            tma_load_2d_pair(sa + L.a_bytes + c * L.b_box, &tm_w, kb * kBK2 + c * kBK,
+                             rank * (p.dg / 2), leader_bar(stage), pol_keep);
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_bf16_f32(2 * kBM, p.dg, false, false);
+      int stage = 0;
+      uint32_t phase = 0, acc = 0, acc_phase = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+        if (!mbar_wait(bar(14 + acc), acc_phase ^ 1, abort_flag, p.status, kDevTimeoutGate)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!(ok = mbar_wait(bar(stage), phase, abort_flag, p.status, kDevTimeoutGate))) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * L.stage_bytes);
+          const uint32_t sb = sa + L.a_bytes;
+#pragma unroll
+          for (int k = 0; k < kBK2 / 16; ++k) {
+            const uint32_t c = k >> 2, kx = (k & 3) * 32;
+            umma_ss_pair(d_tmem, sw128_desc(sa + c * L.a_box + kx, 16, 1024),
+                         sw128_desc(sb + c * L.b_box + kx, 16, 1024), idesc, (kb | k) != 0);
+          }
+          umma_commit_pair(leader_bar(6 + stage));  // both CTAs may refill this stage
+          umma_commit_pair(peer_bar(6 + stage));
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(leader_bar(12 + acc));  // both accumulator halves are ready
+        umma_commit_pair(peer_bar(12 + acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3;
+    const int row_local = quarter * 32 + lane;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+      if (!mbar_wait(bar(12 + acc), acc_phase, abort_flag, p.status, kDevTimeoutGate)) break;
+      tc_fence_after();
+      const uint32_t t_addr =
+          tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
+      float sum = 0.0f;
+      for (int c = 0; c < p.dg; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(t_addr + c, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          sum = fmaf(s_w2[c + j], gelu_erf(__uint_as_float(r[j]) + s_b1[c + j]), sum);
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(leader_bar(14 + acc));
+      const int row = tile * 2 * kBM + static_cast<int>(rank) * kBM + row_local;
+      if (row < p.n) p.z[row] = sum + p.b2;
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no commit or arrival can still target the other CTA
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 }  // namespace
 
 tg_status launch_gate_simt(const void* h, tg_dtype dt, int64_t n, int d, const void* W1,
@@ -250,10 +431,13 @@ tg_status launch_gate_simt(const void* h, tg_dtype dt, int64_t n, int d, const v
 tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const float* b1, int dg,
                          const float* w2, float b2, float* z, cudaStream_t st) {
   CUtensorMap tm_h, tm_w;
+  // CTA-pair kernel (each CTA stages half of W1) when the 128-column stages tile d
+  const bool pairs = num_sms() >= 2 && d % kBK2 == 0;
   if (!encode_tmap_2d_bf16(&tm_h, h, static_cast<uint64_t>(d), static_cast<uint64_t>(n),
                            static_cast<uint64_t>(d) * 2, kBK, kBM) ||
       !encode_tmap_2d_bf16(&tm_w, W1, static_cast<uint64_t>(d), static_cast<uint64_t>(dg),
-                           static_cast<uint64_t>(d) * 2, kBK, static_cast<uint32_t>(dg)))
+                           static_cast<uint64_t>(d) * 2, kBK,
+                           static_cast<uint32_t>(pairs ? dg / 2 : dg)))
     return set_error(TG_ERR_CUDA, "cuTensorMapEncodeTiled failed for the gate operands");
   GateTcParams p;
   p.b1 = b1;
@@ -265,6 +449,20 @@ tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const 
   p.n = static_cast<int32_t>(n);
   p.d = d;
   p.dg = dg;
+  if (pairs) {
+    p.num_tiles = static_cast<int32_t>((n + 2 * kBM - 1) / (2 * kBM));  // 256-row tiles
+    const Gate2Layout L2(dg);
+    const size_t smem2 = L2.total + 1024;
+    tg_status r2 = cuda_check(cudaFuncSetAttribute(gate_tc2_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   static_cast<int>(smem2)),
+                              "gate pair smem attribute");
+    if (r2 != TG_OK) return r2;
+    int npairs = num_sms() / 2;
+    if (npairs > p.num_tiles) npairs = p.num_tiles;
+    gate_tc2_kernel<<<2 * npairs, kThreads, smem2, st>>>(tm_h, tm_w, p);
+    return cuda_check(cudaGetLastError(), "gate_tc2 launch");
+  }
   p.num_tiles = static_cast<int32_t>((n + kBM - 1) / kBM);
   const GateSmemLayout L(dg);
   const size_t smem = L.total + 1024;

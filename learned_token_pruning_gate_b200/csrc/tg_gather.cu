@@ -144,37 +144,56 @@ __global__ void __launch_bounds__(kWarps * 32) gather_kernel(const __grid_consta
       const int hv = p.head_dim / VE;  // vectors per head
       const int hh = hv / 2;           // vectors per half head
       const int n_tasks = g.rope_heads * hh;
-      for (int task = lane; task < n_tasks; task += 32) {
-        const int head = task / hh;
-        const int c = task - head * hh;
-        const int off = head * hv + c;
-        uint4 va = __ldg(src + off);
-        uint4 vb = __ldg(src + off + hh);
+      // four pair-tasks per lane per round: all eight loads are issued before any
+      // rotation or store, so a warp keeps 4 KB of the row in flight
+      constexpr int kU = 4;
+      for (int base = 0; base < n_tasks; base += 32 * kU) {
+        uint4 va[kU], vb[kU];
+        int off[kU], cc[kU];
 #pragma unroll
-        for (int e = 0; e < VE; ++e) {
-          const int a = c * VE + e;
-          const float cs = s_cos[warp][a], sn = s_sin[warp][a];
-          const float x0 = E::get(va, e), x1 = E::get(vb, e);
-          E::set(va, e, x0 * cs - x1 * sn);
-          E::set(vb, e, x1 * cs + x0 * sn);
+        for (int u = 0; u < kU; ++u) {
+          const int task = base + lane + 32 * u;
+          const int head = task / hh;
+          cc[u] = task - head * hh;
+          off[u] = head * hv + cc[u];
+          if (task < n_tasks) {
+            va[u] = __ldg(src + off[u]);
+            vb[u] = __ldg(src + off[u] + hh);
+          }
         }
-        dst[off] = va;
-        dst[off + hh] = vb;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          if (base + lane + 32 * u >= n_tasks) continue;
+#pragma unroll
+          for (int e = 0; e < VE; ++e) {
+            const int a = cc[u] * VE + e;
+            const float cs = s_cos[warp][a], sn = s_sin[warp][a];
+            const float x0 = E::get(va[u], e), x1 = E::get(vb[u], e);
+            E::set(va[u], e, x0 * cs - x1 * sn);
+            E::set(vb[u], e, x1 * cs + x0 * sn);
+          }
+          dst[off[u]] = va[u];
+          dst[off[u] + hh] = vb[u];
+        }
       }
       first_plain = g.rope_heads * hv;
     }
 
-    // Plain copy: four independent 16-byte loads in flight per lane.
-    int vv = first_plain + lane;
-    for (; vv + 96 < g.row_vecs; vv += 128) {
-      uint4 a0 = __ldg(src + vv), a1 = __ldg(src + vv + 32);
-      uint4 a2 = __ldg(src + vv + 64), a3 = __ldg(src + vv + 96);
-      dst[vv] = a0;
-      dst[vv + 32] = a1;
-      dst[vv + 64] = a2;
-      dst[vv + 96] = a3;
+    // Plain copy: eight independent 16-byte loads in flight per lane per round.
+    constexpr int kC = 8;
+    for (int base = first_plain; base < g.row_vecs; base += 32 * kC) {
+      uint4 a[kC];
+#pragma unroll
+      for (int u = 0; u < kC; ++u) {
+        const int vv = base + lane + 32 * u;
+        if (vv < g.row_vecs) a[u] = __ldg(src + vv);
+      }
+#pragma unroll
+      for (int u = 0; u < kC; ++u) {
+        const int vv = base + lane + 32 * u;
+        if (vv < g.row_vecs) dst[vv] = a[u];
+      }
     }
-    for (; vv < g.row_vecs; vv += 32) dst[vv] = __ldg(src + vv);
   }
 }
 
