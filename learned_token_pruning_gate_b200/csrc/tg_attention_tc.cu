@@ -237,24 +237,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         return mbar_wait(b, par, abort_flag, p.status, kDevTimeoutAttn);
       };
       // S_x = Q_x K^T for head x with the K tile in stage s
+      // Descriptors are built once; a k-step or a stage only moves the start
+      // address, which is the low field (address >> 4) of the descriptor, so each
+      // MMA costs one add.  (Shared memory stays below 256 KB: no carry out.)
+      const uint64_t d_q[2] = {sw128_desc(sb + L::kQa, 16, 1024), sw128_desc(sb + L::kQb, 16, 1024)};
+      const uint64_t d_k0 = sw128_desc(sb + L::kK, 16, 1024);
+      const uint64_t d_v0 = sw128_desc(sb + L::kV, L::kBox, 1024);
       auto issue_s = [&](int x, int s) {
-        const uint32_t qb = sb + (x ? L::kQb : L::kQa);
-        const uint32_t kb = sb + L::kK + s * L::kTile;
+        const uint64_t dq = d_q[x];
+        const uint64_t dk = d_k0 + ((s * L::kTile) >> 4);
+        const uint32_t ts = tmem + x * 128;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
-          umma_ss(tmem + x * 128, sw128_desc(qb + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
-                  idesc_qk, kk > 0 ? 1u : 0u);
+          constexpr uint32_t kBox16 = L::kBox >> 4;
+          const uint32_t off = (kk >> 2) * kBox16 + (kk & 3) * 2;
+          umma_ss(ts, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(kSFull + x));
       };
       // O_x (+)= P_x V with the V tile in stage s
       auto issue_pv = [&](int x, int s, bool acc) {
-        const uint32_t vb = sb + L::kV + s * L::kTile;
+        const uint64_t dv = d_v0 + ((s * L::kTile) >> 4);
+        const uint32_t to = tmem + 256 + x * 128, tp = tmem + x * 128;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
-                  sw128_desc(vb + kk * 2048, L::kBox, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          umma_ts(to, tp + kk * 8, dv + kk * (2048 >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
       int rs = 0;
       uint32_t rph = 0, q_waits = 0, p_waits[2] = {0, 0}, of_waits[2] = {0, 0};

@@ -239,11 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // A stage covers 128 columns of the residual (two adjacent 128-byte swizzle boxes
 // per row), so each row contributes 256 contiguous bytes per TMA round.
 constexpr int kStages2 = 3;
+constexpr int kThreads2 = 320;  // TMA warp, MMA warp, 8 epilogue warps (2 per TMEM lane quarter)
 constexpr int kBK2 = 128;
 
 struct Gate2Layout {
   uint32_t stage_bytes, a_bytes, a_box, b_box;
-  uint32_t bars_off, misc_off, b1_off, w2_off, total;
+  uint32_t bars_off, misc_off, b1_off, w2_off, part_off, total;
   __host__ __device__ Gate2Layout(int dg) {
     a_box = kBM * kBK * 2;                             // 128 rows x 64 cols
     b_box = static_cast<uint32_t>(dg / 2) * kBK * 2;   // dg/2 rows x 64 cols
@@ -253,11 +254,12 @@ struct Gate2Layout {
     misc_off = bars_off + 24 * 8;
     b1_off = misc_off + 16;
     w2_off = b1_off + 256 * 4;
-    total = w2_off + 256 * 4;
+    part_off = w2_off + 256 * 4;  // [2 accumulators][128 rows] partial row sums
+    total = part_off + 2 * 128 * 4;
   }
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     gate_tc2_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ GateTcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -287,7 +289,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(12 + a), 1);
-      mbar_init(bar(14 + a), 256);  // both CTAs' epilogue threads
+      mbar_init(bar(14 + a), 512);  // both CTAs' epilogue threads
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -299,7 +301,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_relinquish_pair();
   }
   if (warp >= 2) {
-    for (int i = threadIdx.x - 64; i < p.dg; i += 128) {
+    for (int i = threadIdx.x - 64; i < p.dg; i += 256) {
       s_b1[i] = p.b1[i];
       s_w2[i] = p.w2[i];
     }
@@ -374,8 +376,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
+    // warps 2-5 take the first half of the hidden columns, warps 6-9 the rest
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row_local = quarter * 32 + lane;
+    const int c_split = ((p.dg / 32) / 2) * 32;
+    const int c_lo = half ? c_split : 0, c_hi = half ? p.dg : c_split;
+    float* s_part = reinterpret_cast<float*>(smem + L.part_off);
     uint32_t acc = 0, acc_phase = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs) {
       if (!mbar_wait(bar(12 + acc), acc_phase, abort_flag, p.status, kDevTimeoutGate)) break;
@@ -383,7 +390,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t t_addr =
           tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
       float sum = 0.0f;
-      for (int c = 0; c < p.dg; c += 32) {
+      for (int c = c_lo; c < c_hi; c += 32) {
         uint32_t r[32];
         tmem_ld32(t_addr + c, r);
         tmem_ld_wait(r);
@@ -393,8 +400,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive_cluster(leader_bar(14 + acc));
+      if (half) s_part[acc * 128 + row_local] = sum;
+      named_barrier(1, 256);  // both halves of every row are summed
       const int row = tile * 2 * kBM + static_cast<int>(rank) * kBM + row_local;
-      if (row < p.n) p.z[row] = sum + p.b2;
+      if (!half && row < p.n) p.z[row] = sum + s_part[acc * 128 + row_local] + p.b2;
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -460,7 +469,7 @@ tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const 
     if (r2 != TG_OK) return r2;
     int npairs = num_sms() / 2;
     if (npairs > p.num_tiles) npairs = p.num_tiles;
-    gate_tc2_kernel<<<2 * npairs, kThreads, smem2, st>>>(tm_h, tm_w, p);
+    gate_tc2_kernel<<<2 * npairs, kThreads2, smem2, st>>>(tm_h, tm_w, p);
     return cuda_check(cudaGetLastError(), "gate_tc2 launch");
   }
   p.num_tiles = static_cast<int32_t>((n + kBM - 1) / kBM);
