@@ -61,7 +61,8 @@ typedef enum {
     TG_ERR_ALIGNMENT = 4,    /* a pointer or row pitch is not 16-byte aligned */
     TG_ERR_UNSUPPORTED = 5,  /* valid but outside what the kernels implement */
     TG_ERR_CUDA = 6,         /* a CUDA runtime/driver call or launch failed */
-    TG_ERR_DEVICE_CHECK = 7  /* a kernel reported a failure (see tg_device_status) */
+    TG_ERR_DEVICE_CHECK = 7, /* a kernel reported a failure (see tg_device_status) */
+    TG_ERR_WORKSPACE = 8     /* the workspace given is smaller than the call needs */
 } tg_status;
 
 typedef enum { TG_BF16 = 0, TG_FP32 = 1 } tg_dtype;
@@ -184,13 +185,32 @@ TG_API tg_status tg_compact_gather(const int32_t* kept_idx, int64_t m_total, int
  *   cu_kept_h  host [batch+1] kept-row offsets (M = cu_kept_h[batch])
  *   gain, temp device [n_q_heads] fp32 (temp > 0)
  *   out  device [M, n_q_heads, head_dim], dtype;  lse device [n_q_heads, M] or NULL
+ *   workspace, workspace_bytes
+ *        device scratch owned by the caller, or NULL.  With a workspace the
+ *        tensor-core kernel may split the key range of long query tiles over
+ *        several SMs when the batch is too small to fill the GPU; each chunk's
+ *        partial output is merged in a fixed order, so results do not depend on
+ *        scheduling.  Size it with tg_attention_workspace_bytes (same arguments,
+ *        same device); a smaller non-NULL workspace returns TG_ERR_WORKSPACE.
+ *        16-byte aligned.  Calls that share a workspace must not overlap on the
+ *        GPU (the call clears its counters with an asynchronous memset on stream).
  *   algo tg_algo; the tcgen05 kernel needs bf16 and head_dim in {64, 128}.
  */
 TG_API tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dtype dtype,
                              int32_t batch, const int32_t* cu_kept_h, int32_t n_q_heads,
                              int32_t n_kv_heads, int32_t head_dim, const float* logsig,
                              const float* gain, const float* temp, void* out, float* lse,
-                             int32_t algo, tg_stream_t stream);
+                             void* workspace, size_t workspace_bytes, int32_t algo,
+                             tg_stream_t stream);
+
+/*
+ * Bytes of workspace tg_gated_attention can use for this batch and head shape
+ * on the current device (0 when it would not split, e.g. large batches, fp32,
+ * or TG_ALGO_SIMT).  Host-only: reads cu_kept_h, launches nothing.
+ */
+TG_API tg_status tg_attention_workspace_bytes(tg_dtype dtype, int32_t batch, const int32_t* cu_kept_h,
+                                       int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                       int32_t algo, size_t* bytes_out);
 
 #ifdef __cplusplus
 }

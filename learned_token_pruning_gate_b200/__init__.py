@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "TG_BF16", "TG_FP32", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "TokenGateError",
     "library", "kept_offsets", "gate_score", "topk_select", "compact_gather", "gated_attention",
-    "gated_prefill", "device_status", "EXPORTED_SYMBOLS",
+    "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -37,7 +37,7 @@ LIB_PATH = os.path.join(_HERE, "libtokengate.so")
 EXPORTED_SYMBOLS = (
     "tg_status_string", "tg_last_error_message", "tg_version", "tg_device_status",
     "tg_kept_offsets", "tg_gate_score", "tg_topk_select", "tg_compact_gather",
-    "tg_gated_attention",
+    "tg_gated_attention", "tg_attention_workspace_bytes",
 )
 
 
@@ -81,7 +81,9 @@ def library():
                                     ctypes.POINTER(GatherTensor), _i32, _i32, ctypes.c_double,
                                     _vp, _vp, _vp]
     L.tg_gated_attention.argtypes = [_vp, _vp, _vp, ctypes.c_int, _i32, _i32p, _i32, _i32, _i32,
-                                     _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+                                     _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _i32, _vp]
+    L.tg_attention_workspace_bytes.argtypes = [ctypes.c_int, _i32, _i32p, _i32, _i32, _i32, _i32,
+                                               ctypes.POINTER(ctypes.c_size_t)]
     for name in EXPORTED_SYMBOLS:
         if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -220,12 +222,24 @@ def compact_gather(kept_idx, cu_seqlens, doc_begin, doc_end, budget, tensors, ro
     return outs, logsig_out
 
 
+def attention_workspace_bytes(cu_kept_host, n_q_heads, n_kv_heads, head_dim, dtype="bf16",
+                              algo=ALGO_AUTO):
+    """Workspace bytes tg_gated_attention may use for this batch on the current device."""
+    cu, cu_p = _host_i32(cu_kept_host)
+    code = 0 if dtype in ("bf16", torch.bfloat16) else 1
+    out = ctypes.c_size_t(0)
+    _check("tg_attention_workspace_bytes", library().tg_attention_workspace_bytes(
+        code, len(cu) - 1, cu_p, n_q_heads, n_kv_heads, head_dim, algo, ctypes.byref(out)))
+    return int(out.value)
+
+
 def gated_attention(q, k, v, cu_kept_host, logsig=None, gain=None, temp=None, out=None,
-                    lse=None, algo=ALGO_AUTO, want_lse=False):
+                    lse=None, algo=ALGO_AUTO, want_lse=False, workspace="auto"):
     """Token-gated causal GQA attention over packed kept rows.
 
     q [M, Hq, d], k/v [M, Hkv, d]; cu_kept_host [B+1] host offsets.
-    Returns (out [M, Hq, d], lse [Hq, M] or None).
+    workspace: "auto" (allocate what the call can use), None (no split), or a
+    uint8 device tensor.  Returns (out [M, Hq, d], lse [Hq, M] or None).
     """
     _need_cuda(q, k, v, logsig, gain, temp)
     M, Hq, dh = q.shape
@@ -235,9 +249,14 @@ def gated_attention(q, k, v, cu_kept_host, logsig=None, gain=None, temp=None, ou
         out = torch.empty_like(q)
     if want_lse and lse is None:
         lse = torch.empty((Hq, M), dtype=torch.float32, device=q.device)
+    if isinstance(workspace, str):
+        nbytes = attention_workspace_bytes(cu, Hq, Hkv, dh, q.dtype, algo)
+        workspace = (torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None)
+    ws_bytes = 0 if workspace is None else workspace.numel()
     _check("tg_gated_attention", library().tg_gated_attention(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), len(cu) - 1, cu_p, Hq, Hkv, dh, _ptr(logsig),
-        _ptr(gain), _ptr(temp), _ptr(out), _ptr(lse), algo, _stream(q.device)))
+        _ptr(gain), _ptr(temp), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, algo,
+        _stream(q.device)))
     return out, lse
 
 

@@ -165,6 +165,7 @@ const char* tg_status_string(tg_status s) {
     case TG_ERR_UNSUPPORTED: return "TG_ERR_UNSUPPORTED";
     case TG_ERR_CUDA: return "TG_ERR_CUDA";
     case TG_ERR_DEVICE_CHECK: return "TG_ERR_DEVICE_CHECK";
+    case TG_ERR_WORKSPACE: return "TG_ERR_WORKSPACE";
   }
   return "TG_ERR_UNKNOWN";
 }
@@ -296,11 +297,33 @@ tg_status tg_compact_gather(const int32_t* kept_idx, int64_t m_total, int32_t ba
                        logsig_out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+tg_status tg_attention_workspace_bytes(tg_dtype dtype, int32_t batch, const int32_t* cu_kept_h,
+                                       int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                       int32_t algo, size_t* bytes_out) {
+  if (!bytes_out) return set_error(TG_ERR_INVALID_ARG, "bytes_out is null");
+  *bytes_out = 0;
+  if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
+  PromptTable t;
+  int max_len = 0;
+  tg_status r = build_kept_table(batch, cu_kept_h, &t, &max_len);
+  if (r != TG_OK) return r;
+  if (n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0)
+    return set_error(TG_ERR_SHAPE, "n_q_heads=%d n_kv_heads=%d", n_q_heads, n_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(TG_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", head_dim);
+  if (algo < TG_ALGO_AUTO || algo > TG_ALGO_TCGEN05)
+    return set_error(TG_ERR_INVALID_ARG, "algo %d", algo);
+  if (dtype != TG_BF16 || algo == TG_ALGO_SIMT) return TG_OK;
+  *bytes_out = attn_tc_workspace_bytes(t, n_q_heads, n_kv_heads, head_dim);
+  return TG_OK;
+}
+
 tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dtype dtype,
                              int32_t batch, const int32_t* cu_kept_h, int32_t n_q_heads,
                              int32_t n_kv_heads, int32_t head_dim, const float* logsig,
                              const float* gain, const float* temp, void* out, float* lse,
-                             int32_t algo, tg_stream_t stream) {
+                             void* workspace, size_t workspace_bytes, int32_t algo,
+                             tg_stream_t stream) {
   if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
   PromptTable t;
   int max_len = 0;
@@ -324,8 +347,10 @@ tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dty
   if (algo == TG_ALGO_SIMT || !tc_ok)
     return launch_attn_simt(q, k, v, dtype, t, max_len, n_q_heads, n_kv_heads, head_dim, logsig,
                             gain, temp, out, lse, st);
+  if (workspace && !aligned16(workspace))
+    return set_error(TG_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   return launch_attn_tc(q, k, v, t, max_len, n_q_heads, n_kv_heads, head_dim, logsig, gain, temp,
-                        out, lse, st);
+                        out, lse, workspace, workspace_bytes, st);
 }
 
 }  // extern "C"

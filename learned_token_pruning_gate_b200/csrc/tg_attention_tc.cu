@@ -12,8 +12,13 @@
 // K/V tile is loaded once and feeds two independent softmax warpgroups that
 // take turns with the tensor core (while one computes softmax, the tensor core
 // runs the other's P.V and next Q.K^T).  The kernel is persistent: one CTA per
-// SM walks the items in order of decreasing length (longest first), so the
-// causal imbalance is spread across SMs.
+// SM.  Work units are items, or for small problems chunks of an item's key
+// range, sorted longest first and dealt to the CTAs in boustrophedon order
+// (0..G-1, then G-1..0, ...), which evens out the causal imbalance.  When an
+// item is split, every chunk writes its normalised partial output and
+// log-sum-exp to the caller's workspace; the chunk that finishes last (a
+// counter per item and head, no waiting) merges all partials in chunk order,
+// so the result does not depend on which chunk finishes last.
 //
 //   warp 0     TMA: both Q tiles of an item, then K and V tiles (128 keys)
 //              into a ring of shared-memory stages (128-byte swizzle)
@@ -48,6 +53,9 @@ constexpr int kBN = 128;       // keys per tile
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
+constexpr int kMaxUnits = 2048;  // work units listed explicitly when items are split
+constexpr int kMaxChunks = 4;    // chunks per split item
+
 struct TcParams {
   int32_t kept_start[kMaxBatch + 1];
   int32_t order[kMaxBatch];      // prompts by query-tile count, descending
@@ -65,6 +73,22 @@ struct TcParams {
   int32_t pairs_per_kvh;  // ceil(group / 2)
   int32_t pairs;          // head pairs per (prompt, query tile) = hkv * pairs_per_kvh
   int32_t n_items;
+  int32_t n_units;        // = n_items unless items are split
+  // split items: per slot and head, [DH/4][128] float4 (a warp's rows contiguous),
+  // the rows' log2-domain log-sum-exp, and one arrival counter per item and head
+  float4* part_o;
+  float* part_lse;
+  int32_t* part_cnt;
+};
+
+// Explicit unit list (split plans only): .x item rank, .y = slot << 8 | chunk << 4 | chunks.
+template <bool kSplit>
+struct UnitTable {
+  int32_t unused;
+};
+template <>
+struct UnitTable<true> {
+  int2 unit[kMaxUnits];
 };
 
 template <int DH>
@@ -80,7 +104,7 @@ struct Lay {
   static constexpr uint32_t kBias = kV + kStages * kTile;  // [2 heads][2 parity][128] fp32
   static constexpr uint32_t kBars = kBias + 2 * 2 * 128 * 4;
   static constexpr uint32_t kMisc = kBars + 32 * 8;
-  static constexpr uint32_t kTotal = kMisc + 16;
+  static constexpr uint32_t kTotal = kMisc + 16;  // tmem slot, abort flag, last-chunk flags[2]
   static constexpr uint32_t kDynSmem = kTotal + 1024;
 };
 
@@ -132,16 +156,52 @@ __device__ __forceinline__ Item decode_item(const TcParams& p, int r) {
   return it;
 }
 
+struct Unit {
+  Item it;
+  int j0, j1;     // key tiles [j0, j1) of the item's 0..t
+  int c, n;       // chunk c of n (n = 1: the whole item)
+  int slot;       // first partial slot of a split item
+};
+
+template <bool kSplit>
+__device__ __forceinline__ Unit decode_unit(const TcParams& p, const UnitTable<kSplit>& tab, int u) {
+  Unit w;
+  if constexpr (kSplit) {
+    const int2 e = tab.unit[u];
+    w.it = decode_item(p, e.x);
+    w.n = e.y & 15;
+    w.c = (e.y >> 4) & 15;
+    w.slot = e.y >> 8;
+    const int nkv = w.it.t + 1;
+    w.j0 = w.c * nkv / w.n;
+    w.j1 = (w.c + 1) * nkv / w.n;
+  } else {
+    w.it = decode_item(p, u);
+    w.n = 1;
+    w.c = 0;
+    w.slot = 0;
+    w.j0 = 0;
+    w.j1 = w.it.t + 1;
+  }
+  return w;
+}
+
+// Unit of round k for CTA r of G: boustrophedon order over the sorted units.
+__device__ __forceinline__ int snake_unit(int k, int r, int g) {
+  return k * g + ((k & 1) ? g - 1 - r : r);
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
 
-template <int DH>
+template <int DH, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ TcParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ TcParams p,
+                   const __grid_constant__ UnitTable<kSplit> tab) {
   using L = Lay<DH>;
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -150,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
   float* s_bias = reinterpret_cast<float*>(smem + L::kBias);
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -194,8 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int rs = 0;
       uint32_t rph = 0, q_waits = 0;
       bool ok = true;
-      for (int r = blockIdx.x; ok && r < p.n_items; r += gridDim.x) {
-        const Item it = decode_item(p, r);
+      for (int round = 0; ok; ++round) {
+        const int u = snake_unit(round, blockIdx.x, gridDim.x);
+        if (u >= p.n_units) break;
+        const Unit w = decode_unit<kSplit>(p, tab, u);
+        const Item& it = w.it;
         const int32_t kstart = p.kept_start[it.b];
         if (!(ok = mbar_wait(bar(kQEmpty), (q_waits++ & 1) ^ 1, abort_flag, p.status,
                              kDevTimeoutAttn)))
@@ -208,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(sb + L::kQb + c * L::kBox, &tm_q, it.hb * DH + c * 64,
                         kstart + it.t * kBM, bar(kQFull));
         }
-        for (int j = 0; j <= it.t; ++j) {
+        for (int j = w.j0; j < w.j1; ++j) {
           if (!(ok = mbar_wait(kv_empty(rs), rph ^ 1, abort_flag, p.status, kDevTimeoutAttn)))
             break;
           const int krow = kstart + j * kBN;
@@ -266,9 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       int rs = 0;
       uint32_t rph = 0, q_waits = 0, p_waits[2] = {0, 0}, of_waits[2] = {0, 0};
       bool ok = true;
-      for (int r = blockIdx.x; ok && r < p.n_items; r += gridDim.x) {
-        const Item it = decode_item(p, r);
-        const int n_kv = it.t + 1;
+      for (int round = 0; ok; ++round) {
+        const int u = snake_unit(round, blockIdx.x, gridDim.x);
+        if (u >= p.n_units) break;
+        const Unit w = decode_unit<kSplit>(p, tab, u);
+        const Item& it = w.it;
+        const int n_kv = w.j1 - w.j0;
         if (!(ok = wt(bar(kQFull), q_waits++ & 1))) break;
         if (!(ok = wt(k_full(rs), rph))) break;
         tc_fence_after();
@@ -326,25 +393,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = tmem + lane_off + 256 + x * 128;
     uint32_t s_waits = 0, o_waits = 0, tile_ctr = 0;
     bool ok = true;
-    for (int r = blockIdx.x; ok && r < p.n_items; r += gridDim.x) {
-      const Item it = decode_item(p, r);
+    for (int round = 0; ok; ++round) {
+      const int u = snake_unit(round, blockIdx.x, gridDim.x);
+      if (u >= p.n_units) break;
+      const Unit w = decode_unit<kSplit>(p, tab, u);
+      const Item& it = w.it;
       if (x == 1 && !it.has_b) continue;
       const int head = x ? it.hb : it.ha;
       const int32_t kstart = p.kept_start[it.b];
       const int32_t len = p.kept_start[it.b + 1] - kstart;
-      const int n_kv = it.t + 1;
+      const int n_kv = w.j1 - w.j0;
       const float scale = kLog2e / (sqrtf(static_cast<float>(DH)) * __ldg(p.temp + head));
       const float gl = __ldg(p.gain + head) * kLog2e;
       const float2 sc2 = make_float2(scale, scale);
       float m = -INFINITY, l = 0.0f;
       // this thread's key of the next tile's bias, loaded one tile ahead
-      float next_bias = (p.logsig && rl < len) ? gl * __ldg(p.logsig + kstart + rl) : 0.0f;
+      const int key0 = w.j0 * kBN + rl;
+      float next_bias = (p.logsig && key0 < len) ? gl * __ldg(p.logsig + kstart + key0) : 0.0f;
       for (int j = 0; j < n_kv; ++j) {
+        const int jabs = w.j0 + j;
         float* bias = s_bias + (x * 2 + (tile_ctr & 1)) * 128;
         ++tile_ctr;
         bias[rl] = next_bias;
         if (j + 1 < n_kv) {
-          const int key = (j + 1) * kBN + rl;
+          const int key = (jabs + 1) * kBN + rl;
           next_bias = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
         }
         named_barrier(1 + x, 128);
@@ -361,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // four independent max chains (short dependency chains for two warps per scheduler)
         float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         const float4* b4 = reinterpret_cast<const float4*>(bias);
-        if (j + 1 < n_kv) {
+        if (jabs != it.t) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -462,29 +534,107 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qi = it.t * kBM + rl;
       const float inv = 1.0f / l;
       __nv_bfloat16* out = p.out + (static_cast<int64_t>(kstart + qi) * p.hq + head) * DH;
+      if (!kSplit || w.n == 1) {
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
-        uint32_t orow[32];
-        tmem_ld32(t_o + c * 32, orow);
-        tmem_ld_wait(orow);
-        if (qi < len) {
-          uint32_t pkd[16];
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t orow[32];
+          tmem_ld32(t_o + c * 32, orow);
+          tmem_ld_wait(orow);
+          if (qi < len) {
+            uint32_t pkd[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(orow[2 * e]) * inv,
-                                                      __uint_as_float(orow[2 * e + 1]) * inv);
-            pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
+            for (int e = 0; e < 16; ++e) {
+              __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(orow[2 * e]) * inv,
+                                                        __uint_as_float(orow[2 * e + 1]) * inv);
+              pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
           }
-          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+        }
+        tc_fence_before();
+        mbar_arrive(bar(kOFree + x));
+        if (p.lse && qi < len)
+          p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (m + log2f(l)) * kLn2;
+      } else {
+        // chunk of a split item: store the normalised partial and its log2 LSE
+        constexpr int kV4 = DH / 4;
+        float4* po = p.part_o + static_cast<int64_t>((w.slot + w.c) * 2 + x) * kV4 * 128 + rl;
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t orow[32];
+          tmem_ld32(t_o + c * 32, orow);
+          tmem_ld_wait(orow);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            __stcg(po + (c * 8 + v4) * 128,
+                   make_float4(__uint_as_float(orow[4 * v4]) * inv, __uint_as_float(orow[4 * v4 + 1]) * inv,
+                               __uint_as_float(orow[4 * v4 + 2]) * inv,
+                               __uint_as_float(orow[4 * v4 + 3]) * inv));
+        }
+        __stcg(p.part_lse + ((w.slot + w.c) * 2 + x) * 128 + rl, m + log2f(l));
+        tc_fence_before();
+        mbar_arrive(bar(kOFree + x));
+        // publish, then count arrivals; the last chunk to arrive merges
+        __threadfence();
+        named_barrier(1 + x, 128);
+        if (rl == 0) last_flag[x] = atomicAdd(p.part_cnt + w.slot * 2 + x, 1) == w.n - 1;
+        named_barrier(1 + x, 128);
+        if (last_flag[x]) {
+          __threadfence();
+          float lc[kMaxChunks], wc[kMaxChunks];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int cc = 0; cc < kMaxChunks; ++cc) {
+            lc[cc] = cc < w.n ? __ldcg(p.part_lse + ((w.slot + cc) * 2 + x) * 128 + rl) : -INFINITY;
+            mx = fmaxf(mx, lc[cc]);
+          }
+          float wsum = 0.0f;
+#pragma unroll
+          for (int cc = 0; cc < kMaxChunks; ++cc) {
+            wc[cc] = cc < w.n ? exp2f(lc[cc] - mx) : 0.0f;
+            wsum += wc[cc];
+          }
+          const float winv = 1.0f / wsum;
+#pragma unroll
+          for (int cc = 0; cc < kMaxChunks; ++cc) wc[cc] *= winv;
+          const float4* pb = p.part_o + static_cast<int64_t>(w.slot * 2 + x) * kV4 * 128 + rl;
+          const int64_t slot_stride = 2 * kV4 * 128;
+#pragma unroll 1
+          for (int c = 0; c < DH / 32; ++c) {
+            float acc[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < w.n; ++cc) {
+#pragma unroll
+              for (int v4 = 0; v4 < 8; ++v4) {
+                const float4 a = __ldcg(pb + cc * slot_stride + (c * 8 + v4) * 128);
+                acc[4 * v4] = fmaf(wc[cc], a.x, acc[4 * v4]);
+                acc[4 * v4 + 1] = fmaf(wc[cc], a.y, acc[4 * v4 + 1]);
+                acc[4 * v4 + 2] = fmaf(wc[cc], a.z, acc[4 * v4 + 2]);
+                acc[4 * v4 + 3] = fmaf(wc[cc], a.w, acc[4 * v4 + 3]);
+              }
+            }
+            if (qi < len) {
+              uint32_t pkd[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                __nv_bfloat162 pp = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+                pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4)
+                dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+            }
+          }
+          if (p.lse && qi < len)
+            p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (mx + log2f(wsum)) * kLn2;
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(kOFree + x));
-      if (p.lse && qi < len)
-        p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (m + log2f(l)) * kLn2;
     }
   }
 
@@ -496,38 +646,141 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DH>
-tg_status launch_dh(const void* q, const void* k, const void* v, TcParams& p, int hkv,
-                    cudaStream_t st) {
-  using Ly = Lay<DH>;
-  CUtensorMap tq, tk, tv;
-  const uint64_t M = static_cast<uint64_t>(p.m_total);
-  if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(p.hq) * DH, M,
-                           static_cast<uint64_t>(p.hq) * DH * 2, 64, kBM) ||
-      !encode_tmap_2d_bf16(&tk, k, static_cast<uint64_t>(hkv) * DH, M,
-                           static_cast<uint64_t>(hkv) * DH * 2, 64, kBN) ||
-      !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(hkv) * DH, M,
-                           static_cast<uint64_t>(hkv) * DH * 2, 64, kBN))
-    return set_error(TG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q/k/v");
-  tg_status r = cuda_check(cudaFuncSetAttribute(attn_tc_kernel<DH>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                static_cast<int>(Ly::kDynSmem)),
-                           "attn smem attribute");
-  if (r != TG_OK) return r;
-  int grid = num_sms();
-  if (grid > p.n_items) grid = p.n_items;
-  attn_tc_kernel<DH><<<grid, kThreads, Ly::kDynSmem, st>>>(tq, tk, tv, p);
-  return cuda_check(cudaGetLastError(), "attn_tc launch");
+// ---------------------------------------------------------------------------
+// Host: work plan.  Items are enumerated in the kernel's rank order (query-tile
+// level descending, prompts longest first, head pairs); an item at level t has
+// t + 1 key tiles.  For k = 1..kMaxChunks chunks of the longest item, items
+// longer than C = ceil(max / k) tiles are cut into ceil(n / C) chunks; the plan
+// with the smallest modelled makespan under the kernel's boustrophedon deal
+// wins (a split must gain at least 3 % to be taken).  Cost model, in key
+// tiles: a unit costs its tiles plus 0.3 (Q load, epilogue), a chunk of a
+// split item 1.0 more (partial store and merge).
+// ---------------------------------------------------------------------------
+struct AttnPlan {
+  int grid = 0;
+  int n_units = 0;
+  int n_slots = 0;
+  bool split = false;
+  size_t workspace = 0;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static size_t split_workspace_bytes(int n_slots, int dh) {
+  return align256(static_cast<size_t>(n_slots) * 2 * sizeof(int32_t)) +
+         align256(static_cast<size_t>(n_slots) * 2 * 128 * sizeof(float)) +
+         static_cast<size_t>(n_slots) * 2 * 128 * dh * sizeof(float);
 }
 
-}  // namespace
+static void item_lengths(const TcParams& p, int32_t* nkv) {
+  int r = 0;
+  for (int t = p.nt_sorted[0] - 1; t >= 0; --t)
+    for (int k = 0; k < p.batch && p.nt_sorted[k] > t; ++k)
+      for (int pr = 0; pr < p.pairs; ++pr) nkv[r++] = t + 1;
+}
 
-tg_status launch_attn_tc(const void* q, const void* k, const void* v, const PromptTable& pt,
-                         int max_len, int hq, int hkv, int dh, const float* logsig,
-                         const float* gain, const float* temp, void* out, float* lse,
-                         cudaStream_t st) {
-  (void)max_len;
-  TcParams p;
+static double snake_makespan(const double* cost_sorted, int n, int g, double* load) {
+  for (int i = 0; i < g; ++i) load[i] = 0.0;
+  for (int i = 0; i < n; ++i) {
+    const int k = i / g, r = i - k * g;
+    load[(k & 1) ? g - 1 - r : r] += cost_sorted[i];
+  }
+  double mx = 0.0;
+  for (int i = 0; i < g; ++i) mx = load[i] > mx ? load[i] : mx;
+  return mx;
+}
+
+// Fills `tab` (when non-null and the plan splits) and returns the plan.
+static AttnPlan make_plan(const TcParams& p, int dh, int n_sms, bool allow_split,
+                          UnitTable<true>* tab) {
+  constexpr double kOverhead = 0.3, kChunkCost = 1.0;
+  AttnPlan best;
+  best.n_units = p.n_items;
+  best.grid = p.n_items < n_sms ? p.n_items : n_sms;
+  if (!allow_split || p.n_items > kMaxUnits || p.n_items == 0) return best;
+  const int n = p.n_items;
+  int32_t nkv[kMaxUnits];
+  item_lengths(p, nkv);
+  const int max_n = nkv[0];
+  // unit lists for one candidate: (cost, item, chunk, chunks)
+  struct U {
+    double cost;
+    int item, c, s;
+  };
+  static thread_local U units[kMaxUnits], sorted[kMaxUnits];
+  static thread_local double costs[kMaxUnits], load[1024];
+  const int g_cap = n_sms < 1024 ? n_sms : 1024;
+  double base = 0.0;
+  double best_span = 0.0;
+  for (int k = 1; k <= kMaxChunks; ++k) {
+    const int C = (max_n + k - 1) / k;
+    if (k > 1 && C == (max_n + k - 2) / (k - 1)) continue;
+    int nu = 0;
+    bool fits = true;
+    for (int i = 0; i < n && fits; ++i) {
+      const int s = (nkv[i] + C - 1) / C;
+      if (nu + s > kMaxUnits) {
+        fits = false;
+        break;
+      }
+      for (int c = 0; c < s; ++c) {
+        const int lo = c * nkv[i] / s, hi = (c + 1) * nkv[i] / s;
+        units[nu++] = {hi - lo + kOverhead + (s > 1 ? kChunkCost : 0.0), i, c, s};
+      }
+    }
+    if (!fits) continue;
+    // stable sort by cost, descending (insertion into runs: costs take few values)
+    int m = 0;
+    for (int i = 0; i < nu; ++i) {
+      int j = m++;
+      while (j > 0 && sorted[j - 1].cost < units[i].cost) {
+        sorted[j] = sorted[j - 1];
+        --j;
+      }
+      sorted[j] = units[i];
+    }
+    for (int i = 0; i < nu; ++i) costs[i] = sorted[i].cost;
+    const int g = nu < g_cap ? nu : g_cap;
+    const double span = snake_makespan(costs, nu, g, load);
+    if (k == 1) {
+      base = best_span = span;
+      continue;
+    }
+    if (span < best_span && span < 0.97 * base) {
+      best_span = span;
+      best.n_units = nu;
+      best.grid = g;
+      best.split = true;
+      if (tab) {
+        int slot = 0;
+        // slots: consecutive per split item, in item order
+        static thread_local int32_t item_slot[kMaxUnits];
+        for (int i = 0; i < n; ++i) item_slot[i] = -1;
+        for (int i = 0; i < nu; ++i)
+          if (units[i].s > 1 && units[i].c == 0) {
+            item_slot[units[i].item] = slot;
+            slot += units[i].s;
+          }
+        for (int i = 0; i < nu; ++i) {
+          const U& e = sorted[i];
+          const int sl = e.s > 1 ? item_slot[e.item] : 0;
+          tab->unit[i] = make_int2(e.item, (sl << 8) | (e.c << 4) | e.s);
+        }
+        best.n_slots = slot;
+      } else {
+        int slot = 0;
+        for (int i = 0; i < nu; ++i)
+          if (units[i].s > 1 && units[i].c == 0) slot += units[i].s;
+        best.n_slots = slot;
+      }
+    }
+  }
+  if (best.split) best.workspace = split_workspace_bytes(best.n_slots, dh);
+  return best;
+}
+
+static tg_status fill_params(const PromptTable& pt, int hq, int hkv, TcParams* pp) {
+  TcParams& p = *pp;
   memset(&p, 0, sizeof(p));
   p.batch = pt.batch;
   for (int b = 0; b <= pt.batch; ++b) p.kept_start[b] = pt.kept_start[b];
@@ -551,24 +804,85 @@ tg_status launch_attn_tc(const void* q, const void* k, const void* v, const Prom
     p.nt_sorted[i] = nt[p.order[i]];
     tiles += p.nt_sorted[i];
   }
-  p.logsig = logsig;
-  p.gain = gain;
-  p.temp = temp;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.status = device_status_word();
-  if (!p.status) return set_error(TG_ERR_CUDA, "device status word unavailable");
   p.m_total = pt.kept_start[pt.batch];
   p.hq = hq;
   p.group = hq / hkv;
   p.pairs_per_kvh = (p.group + 1) / 2;
   p.pairs = hkv * p.pairs_per_kvh;
   const int64_t n_items = tiles * p.pairs;
-  if (n_items == 0) return TG_OK;
   if (n_items > 0x7FFFFFFF) return set_error(TG_ERR_UNSUPPORTED, "too many attention tiles");
   p.n_items = static_cast<int32_t>(n_items);
-  if (dh == 64) return launch_dh<64>(q, k, v, p, hkv, st);
-  return launch_dh<128>(q, k, v, p, hkv, st);
+  p.n_units = p.n_items;
+  return TG_OK;
+}
+
+template <int DH, bool kSplit>
+tg_status launch_dh(const void* q, const void* k, const void* v, const TcParams& p,
+                    const UnitTable<kSplit>& tab, int grid, int hkv, cudaStream_t st) {
+  using Ly = Lay<DH>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t M = static_cast<uint64_t>(p.m_total);
+  if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(p.hq) * DH, M,
+                           static_cast<uint64_t>(p.hq) * DH * 2, 64, kBM) ||
+      !encode_tmap_2d_bf16(&tk, k, static_cast<uint64_t>(hkv) * DH, M,
+                           static_cast<uint64_t>(hkv) * DH * 2, 64, kBN) ||
+      !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(hkv) * DH, M,
+                           static_cast<uint64_t>(hkv) * DH * 2, 64, kBN))
+    return set_error(TG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q/k/v");
+  tg_status r = cuda_check(cudaFuncSetAttribute(attn_tc_kernel<DH, kSplit>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(Ly::kDynSmem)),
+                           "attn smem attribute");
+  if (r != TG_OK) return r;
+  attn_tc_kernel<DH, kSplit><<<grid, kThreads, Ly::kDynSmem, st>>>(tq, tk, tv, p, tab);
+  return cuda_check(cudaGetLastError(), "attn_tc launch");
+}
+
+}  // namespace
+
+size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh) {
+  TcParams p;
+  if (fill_params(pt, hq, hkv, &p) != TG_OK || p.n_items == 0) return 0;
+  return make_plan(p, dh, num_sms(), true, nullptr).workspace;
+}
+
+tg_status launch_attn_tc(const void* q, const void* k, const void* v, const PromptTable& pt,
+                         int max_len, int hq, int hkv, int dh, const float* logsig,
+                         const float* gain, const float* temp, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  (void)max_len;
+  TcParams p;
+  tg_status r = fill_params(pt, hq, hkv, &p);
+  if (r != TG_OK) return r;
+  if (p.n_items == 0) return TG_OK;
+  p.logsig = logsig;
+  p.gain = gain;
+  p.temp = temp;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  static thread_local UnitTable<true> tab;
+  const AttnPlan plan = make_plan(p, dh, num_sms(), workspace != nullptr, &tab);
+  if (plan.split && workspace_bytes < plan.workspace)
+    return set_error(TG_ERR_WORKSPACE, "attention workspace: %zu bytes given, %zu needed",
+                     workspace_bytes, plan.workspace);
+  p.status = device_status_word();
+  if (!p.status) return set_error(TG_ERR_CUDA, "device status word unavailable");
+  if (!plan.split) {
+    const UnitTable<false> none{0};
+    if (dh == 64) return launch_dh<64, false>(q, k, v, p, none, plan.grid, hkv, st);
+    return launch_dh<128, false>(q, k, v, p, none, plan.grid, hkv, st);
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t cnt_bytes = align256(static_cast<size_t>(plan.n_slots) * 2 * sizeof(int32_t));
+  const size_t lse_bytes = align256(static_cast<size_t>(plan.n_slots) * 2 * 128 * sizeof(float));
+  p.part_cnt = reinterpret_cast<int32_t*>(ws);
+  p.part_lse = reinterpret_cast<float*>(ws + cnt_bytes);
+  p.part_o = reinterpret_cast<float4*>(ws + cnt_bytes + lse_bytes);
+  p.n_units = plan.n_units;
+  r = cuda_check(cudaMemsetAsync(p.part_cnt, 0, cnt_bytes, st), "attention workspace counters");
+  if (r != TG_OK) return r;
+  if (dh == 64) return launch_dh<64, true>(q, k, v, p, tab, plan.grid, hkv, st);
+  return launch_dh<128, true>(q, k, v, p, tab, plan.grid, hkv, st);
 }
 
 }  // namespace tg

@@ -57,7 +57,9 @@ tg_status launch_attn_simt(const void* q, const void* k, const void* v, tg_dtype
 tg_status launch_attn_tc(const void* q, const void* k, const void* v, const PromptTable& pt,
                          int max_len, int hq, int hkv, int dh, const float* logsig,
                          const float* gain, const float* temp, void* out, float* lse,
-                         cudaStream_t st);
+                         void* workspace, size_t workspace_bytes, cudaStream_t st);
+// Workspace the tensor-core attention uses to split long items on this device (0 = none).
+size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh);
 
 // Tensor map encoding through the driver entry point (no libcuda link).
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
@@ -269,6 +271,41 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | (static_cast<uint32_t>(b_mn_major) << 16)  // B major
          | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// ---- bulk (non-tensor) copies ---------------------------------------------------
+// global -> shared, completion counted on an mbarrier of this CTA (16-byte aligned,
+// size a multiple of 16)
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// shared -> global, tracked by the issuing thread's bulk async-groups
+__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// wait until at most N committed groups still read their shared-memory source
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// make generic-proxy shared-memory writes visible to the async proxy (bulk copies)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---- CTA pairs (tcgen05 cta_group::2) ----------------------------------------

@@ -13,7 +13,8 @@ import ctypes
 import numpy as np
 import torch
 
-from . import (ALGO_AUTO, GatherTensor, _check, _dtype_code, _host_i32, kept_offsets, library)
+from . import (ALGO_AUTO, GatherTensor, _check, _dtype_code, _host_i32,
+               attention_workspace_bytes, kept_offsets, library)
 
 
 class GatedLayer:
@@ -48,6 +49,9 @@ class GatedLayer:
         self.logsig = torch.empty(max(self.M, 1), **f32)
         self.out = torch.empty_like(self.q_c)
         self.lse = torch.empty((self.Hq, self.M), **f32) if want_lse else None
+        ws = attention_workspace_bytes(self.cu_kept_host, self.Hq, self.Hkv, self.dh, q.dtype, algo)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
+        self.ws_bytes = ws
         self.dcode = _dtype_code(h)
         self.tensors = (GatherTensor * 4)()
         for i, (src, dst, heads) in enumerate([(h, self.h_c, 0), (q, self.q_c, self.Hq),
@@ -61,6 +65,7 @@ class GatedLayer:
             h=h, q=q, k=k, v=v, W1=W1, b1=b1, w2=w2, gain=gain, temp=temp, z=self.z,
             kept=self.kept_idx, cu_kept=self.cu_kept, q_c=self.q_c, k_c=self.k_c, v_c=self.v_c,
             logsig=self.logsig, out=self.out).items()}
+        self._p["ws"] = vp(self.workspace.data_ptr()) if self.workspace is not None else None
         self._p["lse"] = vp(self.lse.data_ptr()) if self.lse is not None else None
 
     # each step is one C-ABI call; `stream` is a raw cudaStream_t handle
@@ -86,7 +91,8 @@ class GatedLayer:
         p = self._p
         _check("tg_gated_attention", self.L.tg_gated_attention(
             p["q_c"], p["k_c"], p["v_c"], self.dcode, self.B, self.ck_p, self.Hq, self.Hkv,
-            self.dh, p["logsig"], p["gain"], p["temp"], p["out"], p["lse"], self.algo, stream))
+            self.dh, p["logsig"], p["gain"], p["temp"], p["out"], p["lse"], p["ws"], self.ws_bytes,
+            self.algo, stream))
 
     STAGES = ("gate", "topk", "gather", "attention")
 

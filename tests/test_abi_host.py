@@ -15,6 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "tokengate.h")
 
 OK, INVALID, SHAPE, DTYPE, ALIGN, UNSUP, CUDA = 0, 1, 2, 3, 4, 5, 6
+WORKSPACE = 8
 FAKE = ctypes.c_void_p(0x10000)      # aligned, never dereferenced by a rejected call
 FAKE_ODD = ctypes.c_void_p(0x10008)  # 8-byte aligned only
 
@@ -140,14 +141,58 @@ def test_gather_validation(L):
 def test_attention_validation(L):
     _, ck = _arr([0, 100])
     a = L.tg_gated_attention
-    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 6, 128, None, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
-    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 8, 96, None, FAKE, FAKE, FAKE, None, 0, None) == UNSUP
-    assert a(FAKE, FAKE, FAKE, 1, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, 2, None) == UNSUP
-    assert a(FAKE_ODD, FAKE, FAKE, 0, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, 0,
+    n = None  # workspace pointer
+    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 6, 128, None, FAKE, FAKE, FAKE, None, n, 0, 0,
+             None) == SHAPE
+    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 8, 96, None, FAKE, FAKE, FAKE, None, n, 0, 0,
+             None) == UNSUP
+    assert a(FAKE, FAKE, FAKE, 1, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, n, 0, 2,
+             None) == UNSUP
+    assert a(FAKE_ODD, FAKE, FAKE, 0, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, n, 0, 0,
              None) == ALIGN
+    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, FAKE_ODD,
+             1 << 20, 0, None) == ALIGN
     _, bad = _arr([0, 100, 50])
-    assert a(FAKE, FAKE, FAKE, 0, 2, bad, 16, 8, 128, None, FAKE, FAKE, FAKE, None, 0,
+    assert a(FAKE, FAKE, FAKE, 0, 2, bad, 16, 8, 128, None, FAKE, FAKE, FAKE, None, n, 0, 0,
              None) == INVALID
+
+
+def _ws_bytes(L, cu, hq=16, hkv=8, dh=128, dtype=0, algo=0):
+    _, ck = _arr(cu)
+    out = ctypes.c_size_t(123)
+    st = L.tg_attention_workspace_bytes(dtype, len(cu) - 1, ck, hq, hkv, dh, algo,
+                                        ctypes.byref(out))
+    return st, out.value
+
+
+def test_attention_workspace_plan(L):
+    """The split plan is host logic: small batches that cannot fill the GPU ask
+    for workspace; long prompts, fp32 and the CUDA-core kernel ask for none.
+    (Without a GPU the planner assumes 148 SMs.)"""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("plan sizes below assume 148 SMs")
+    st, b = _ws_bytes(L, [0, 2304])  # one 16k-token prompt kept down to 2304 rows
+    assert st == 0 and b > 0
+    # every partial slot holds 2 heads x 128 rows x (head_dim + 1) floats, plus counters
+    assert b % 4 == 0 and b >= 2 * 128 * 129 * 4
+    st, b = _ws_bytes(L, [0, 8448])  # 66 query tiles x 8 head pairs: no split
+    assert (st, b) == (0, 0)
+    assert _ws_bytes(L, [0, 2304], dtype=1) == (0, 0)  # fp32: CUDA-core kernel
+    assert _ws_bytes(L, [0, 2304], algo=1) == (0, 0)
+    assert _ws_bytes(L, [0, 0]) == (0, 0)  # nothing kept
+    assert _ws_bytes(L, [0, 2304], hkv=6)[0] == SHAPE
+    assert _ws_bytes(L, [0, 2304], dh=96)[0] == UNSUP
+    _, ck = _arr([0, 10])
+    assert L.tg_attention_workspace_bytes(0, 1, ck, 16, 8, 128, 0, None) == INVALID
+    # a workspace smaller than the plan needs is refused before anything launches
+    st, need = _ws_bytes(L, [0, 2304])
+    _, ck = _arr([0, 2304])
+    a = L.tg_gated_attention
+    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, FAKE,
+             need - 16, 0, None) == WORKSPACE
+    assert b"needed" in L.tg_last_error_message()
 
 
 def test_no_gpu_means_cuda_error_not_crash(L):

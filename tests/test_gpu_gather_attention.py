@@ -64,10 +64,11 @@ def test_gather_varlen_small_and_empty(oracle):
 
 # ---- attention -----------------------------------------------------------------
 
-def _attn_case(oracle, lens, Hq, Hkv, dh, dtype, algo, bias=True, seed=0, rows=None):
+def _attn_case(oracle, lens, Hq, Hkv, dh, dtype, algo, bias=True, seed=0, rows=None,
+               workspace="auto"):
     cu, q, k, v, ls, gain, temp = gen.attention_inputs(lens, Hq, Hkv, dh, seed, dtype, bias)
     out, lse = tg.gated_attention(dev(q), dev(k), dev(v), cu, dev(ls), dev(gain), dev(temp),
-                                  algo=algo, want_lse=True)
+                                  algo=algo, want_lse=True, workspace=workspace)
     ref, ref_lse = oracle.gated_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
                                           cu, None if ls is None else ls.numpy(), gain.numpy(),
                                           temp.numpy(), rows=rows)
@@ -84,6 +85,35 @@ def _attn_case(oracle, lens, Hq, Hkv, dh, dtype, algo, bias=True, seed=0, rows=N
 @pytest.mark.parametrize("algo", [tg.ALGO_TCGEN05, tg.ALGO_SIMT])
 def test_attention_bf16_d128(oracle, lens, algo):
     _attn_case(oracle, lens, 16, 8, 128, "bf16", algo, seed=len(lens) + sum(lens))
+
+
+@pytest.mark.parametrize("lens", [[1000], [2304], [5, 0, 260, 1, 640]])
+def test_attention_without_workspace(oracle, lens):
+    """No workspace: every query tile stays on one SM (no key-range split)."""
+    _attn_case(oracle, lens, 16, 8, 128, "bf16", tg.ALGO_TCGEN05, seed=sum(lens) + 3,
+               workspace=None)
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,dh", [([2304], 16, 8, 128), ([1280], 16, 8, 128),
+                                            ([700, 90, 1500], 12, 4, 128), ([900], 4, 2, 64)])
+def test_attention_split_matches_unsplit_and_repeats(lens, Hq, Hkv, dh):
+    """Small batches split long query tiles over several SMs; the merged result
+    must agree with the unsplit kernel and be identical on repeated calls (the
+    merge order is fixed, and each call re-arms the workspace counters)."""
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    need = tg.attention_workspace_bytes(cu, Hq, Hkv, dh)
+    assert need > 0, "this shape is expected to split"
+    cu, q, k, v, ls, gain, temp = gen.attention_inputs(lens, Hq, Hkv, dh, 17, "bf16", True)
+    args = [dev(x) for x in (q, k, v)] + [cu, dev(ls), dev(gain), dev(temp)]
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device="cuda")  # counters must be re-armed
+    o1, l1 = tg.gated_attention(*args, algo=tg.ALGO_TCGEN05, want_lse=True, workspace=ws)
+    o2, l2 = tg.gated_attention(*args, algo=tg.ALGO_TCGEN05, want_lse=True, workspace=ws)
+    o0, l0 = tg.gated_attention(*args, algo=tg.ALGO_TCGEN05, want_lse=True, workspace=None)
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1, l2)
+    assert_close("split vs unsplit", host_f32(o1), host_f32(o0), 2 ** -7, 2 ** -7)
+    assert_close("split vs unsplit lse", l1.cpu().numpy(), l0.cpu().numpy(), 1e-4, 1e-6)
 
 
 @pytest.mark.parametrize("lens,bias", [([700], True), ([700], False), ([64, 200, 3], True)])
