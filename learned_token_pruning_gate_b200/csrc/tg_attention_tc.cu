@@ -117,6 +117,7 @@ enum {
   kOFull = 6,   // [2]
   kOFree = 8,   // [2]
   kKFull = 10,  // [stages]
+  kDrain = 31,  // MMA completion on the way out after an abort
 };
 
 struct Item {
@@ -233,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(v_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
+    mbar_init(bar(kDrain), 1);
     *abort_flag = 0;
     mbar_fence_init();
     prefetch_tmap(&tm_q);
@@ -248,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  int q_loads = 0, tiles_loaded = 0;  // producer thread: loads issued (for the abort drain)
   if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -265,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              kDevTimeoutAttn)))
           break;
         mbar_arrive_expect_tx(bar(kQFull), L::kTile * (it.has_b ? 2 : 1));
+        ++q_loads;
         for (uint32_t c = 0; c < L::kChunks; ++c) {
           tma_load_2d(sb + L::kQa + c * L::kBox, &tm_q, it.ha * DH + c * 64, kstart + it.t * kBM,
                       bar(kQFull));
@@ -276,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(kv_empty(rs), rph ^ 1, abort_flag, p.status, kDevTimeoutAttn)))
             break;
           const int krow = kstart + j * kBN;
+          ++tiles_loaded;
           mbar_arrive_expect_tx(k_full(rs), L::kTile);
           for (uint32_t c = 0; c < L::kChunks; ++c)
             tma_load_2d(sb + L::kK + rs * L::kTile + c * L::kBox, &tm_k, it.hk * DH + c * 64, krow,
@@ -419,10 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int key = (jabs + 1) * kBN + rl;
           next_bias = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
         }
-        named_barrier(1 + x, 128);
-        if (!(ok = mbar_wait(bar(kSFull + x), s_waits++ & 1, abort_flag, p.status,
-                             kDevTimeoutAttn)))
+        ok = mbar_wait(bar(kSFull + x), s_waits++ & 1, abort_flag, p.status, kDevTimeoutAttn);
+        // one outcome for the whole warpgroup (and the bias row is visible)
+        if (named_barrier_or(1 + x, 128, !ok)) {
+          ok = false;
           break;
+        }
         tc_fence_after();
         uint32_t sr[4][32];
 #pragma unroll
@@ -527,9 +534,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O / l
-      if (!(ok = mbar_wait(bar(kOFull + x), o_waits++ & 1, abort_flag, p.status,
-                           kDevTimeoutAttn)))
+      ok = mbar_wait(bar(kOFull + x), o_waits++ & 1, abort_flag, p.status, kDevTimeoutAttn);
+      if (named_barrier_or(1 + x, 128, !ok)) {
+        ok = false;
         break;
+      }
       tc_fence_after();
       const int qi = it.t * kBM + rl;
       const float inv = 1.0f / l;
@@ -640,6 +649,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // a wait gave up: let the loads and MMAs already issued finish (bounded)
+    // before the shared memory and TMEM are released
+    if (warp == 0 && lane == 0) {
+      if (q_loads > 0) mbar_drain(bar(kQFull), (q_loads - 1) & 1);
+      for (int s = 0; s < S && s < tiles_loaded; ++s) {
+        const uint32_t par = ((tiles_loaded - 1 - s) / S) & 1;
+        mbar_drain(k_full(s), par);
+        mbar_drain(v_full(s), par);
+      }
+    }
+    if (warp == 1 && lane == 0) {
+      umma_commit(bar(kDrain));
+      mbar_drain(bar(kDrain), 0);
+    }
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

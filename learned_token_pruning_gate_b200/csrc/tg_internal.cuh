@@ -31,6 +31,7 @@ enum : uint32_t {
   kDevTimeoutAttn = 1u << 1,
   kDevTopkOverflow = 1u << 2,   // selection produced more rows than M_b (skipped)
   kDevGatherIndex = 1u << 3,    // a kept index outside the prompt batch (row skipped)
+  kDevTimeoutGather = 1u << 4,
 };
 
 // Host side: error reporting and the device status word.
@@ -90,6 +91,10 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
+}
+// Raise the barrier's expected transaction bytes without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -370,6 +375,27 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// Named barrier that also ORs a predicate over the participating threads, so a
+// group leaves a loop together when any of its threads gave up waiting.
+__device__ __forceinline__ bool named_barrier_or(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+// Bounded wait that ignores the abort flag: used only on the way out after an
+// abort, so copies or MMAs already issued land before the CTA exits.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < kWaitLimitNs) {
+  }
 }
 
 __device__ __forceinline__ float exp2_approx(float x) {
