@@ -18,6 +18,8 @@
 // cos/sin in fp32 in shared memory, and rotates every head in fp32.  The warp
 // handling tensor 0 of a row also writes the row's bias term
 // l = log sigmoid(z) (0 for question tokens).
+#include <cmath>
+
 #include "tg_internal.cuh"
 
 namespace tg {
@@ -227,11 +229,14 @@ struct BulkParams {
   int32_t row_bytes[TG_MAX_GATHER_TENSORS];
   int32_t row_off[TG_MAX_GATHER_TENSORS];  // offset of the tensor's row inside a batch row
   int32_t rope_heads[TG_MAX_GATHER_TENSORS];
+  // RoPE angle of position pos, dim i: pos * theta^(-2i/d) radians, kept as a
+  // fraction of a turn in 0.64 fixed point (evaluated on the host in fp64): the
+  // product with an integer position, mod 2^64, is the angle's fractional turn
+  uint64_t turns[kMaxHalf];
   const int32_t* kept_idx;
   const float* z;
   float* logsig;
   uint32_t* status;
-  double theta;
   int32_t m_total;
   int32_t n_tensors;
   int32_t head_dim;
@@ -243,7 +248,6 @@ struct BulkParams {
 struct BulkSmem {
   uint8_t stage[kBulkStages][kStageBytes];
   float2 cs[kGroups][kMaxAngles];  // (cos, sin) of each group's batch
-  uint64_t turns[kMaxHalf];        // theta^(-2i/d) / (2 pi) in 0.64 fixed point
   int32_t idx[kIdxCap];            // this CTA's kept indices, batch after batch
   int32_t src_row[kBulkStages][kMaxBatchRows];  // -1: invalid index, row skipped
   int32_t prompt[kBulkStages][kMaxBatchRows];
@@ -276,15 +280,6 @@ __global__ void __launch_bounds__(kBulkThreads, 1) gather_bulk_kernel(const __gr
     const int64_t i = static_cast<int64_t>(blockIdx.x + kb * static_cast<int>(gridDim.x)) * p.rows + r;
     if ((blockIdx.x + kb * static_cast<int>(gridDim.x)) < p.n_batches && i < p.m_total)
       sm.idx[j] = __ldg(p.kept_idx + i);
-  }
-  // RoPE angle of position pos, dim i: pos * theta^(-2i/d) radians.  Kept as a
-  // fraction of a turn in 0.64 fixed point: the product with an integer
-  // position, mod 2^64, is the angle's fractional turn, exact to ~1e-19 turns
-  // times pos (the fixed-point rounding) -- no fp64 work per angle.
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double f = pow(p.theta, -2.0 * static_cast<double>(i) / static_cast<double>(p.head_dim)) *
-                     0.15915494309189535;  // 1 / (2 pi)
-    sm.turns[i] = static_cast<uint64_t>(ldexp(f, 64));
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBulkStages; ++s) {
@@ -407,7 +402,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) gather_bulk_kernel(const __gr
           float sn = 0.0f, c = 1.0f;
           if (src >= 0) {
             const uint32_t pos = static_cast<uint32_t>(src - sm.start[sm.prompt[s][r]]);
-            const uint64_t f = sm.turns[i];
+            const uint64_t f = p.turns[i];
             // top 32 bits of pos * f mod 2^64: the angle's fractional turn
             const uint32_t top = pos * static_cast<uint32_t>(f >> 32) + __umulhi(pos, static_cast<uint32_t>(f));
             // as a signed fraction of a half turn in [-1, 1): angle = pi * x
@@ -530,11 +525,15 @@ tg_status launch_gather(const int32_t* kept_idx, int64_t m_total, const PromptTa
     if (rows > kGroupThreads) rows = kGroupThreads;  // one thread per row writes the bias term
     if (n_tensors > 0 && rows >= 1 && m_total < (int64_t(1) << 31)) {
       b.pt = pt;
+      for (int i = 0; i < half && i < kMaxHalf; ++i) {
+        const double f = std::pow(theta, -2.0 * i / static_cast<double>(p.head_dim)) /
+                         (2.0 * 3.14159265358979323846);
+        b.turns[i] = static_cast<uint64_t>(std::ldexp(f, 64));  // f < 1: fits
+      }
       b.kept_idx = kept_idx;
       b.z = z;
       b.logsig = logsig;
       b.status = p.status;
-      b.theta = theta;
       b.m_total = static_cast<int32_t>(m_total);
       b.n_tensors = n_tensors;
       b.head_dim = p.head_dim;
