@@ -673,16 +673,481 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Pair kernel (tcgen05 cta_group::2, head_dim 128, even GQA groups).
+//
+// A cluster of two CTAs takes one work unit: CTA 0 the unit's head a, CTA 1
+// head b; the two query tiles form the M = 256 rows of every MMA.  Both heads
+// read the same K and V tiles, so each CTA stages only half of them (K: 64 of
+// the 128 keys, V: 64 of the 128 dims) and the pair's MMAs read the other half
+// from the peer: per SM, Q.K^T reads 6 KB instead of 8 KB of shared memory per
+// k-step.  With one head per CTA, TMEM holds two S buffers (2 x 128 columns)
+// next to O (128), so Q.K^T of the next tiles runs while the softmax of the
+// current one does.
+//
+//   warp 0     TMA (each CTA): its Q tile, its halves of K and V tiles into
+//              two rings; the bytes of both CTAs are counted on CTA 0's barriers
+//   warp 1     CTA 0 only: TMEM allocation for the pair and the single MMA
+//              issuer: S(0) S(1) | P(j).V_j S(j+2) | ...; commits go to the
+//              barriers of both CTAs
+//   warps 2-5  softmax of this CTA's head, one query row per thread, and the
+//              epilogue (as in the single-CTA kernel)
+// ---------------------------------------------------------------------------
+constexpr int kPairThreads = 192;
+constexpr int kPKStages = 5, kPVStages = 5;
+
+struct PairLay {
+  static constexpr uint32_t kQBox = kBM * 128;          // 128 rows x 64 bf16
+  static constexpr uint32_t kQ = 0;                     // 2 boxes (dims 0-63, 64-127)
+  static constexpr uint32_t kKBox = 64 * 128;           // 64 keys x 64 bf16
+  static constexpr uint32_t kKStage = 2 * kKBox;        // this CTA's 64 keys, all dims
+  static constexpr uint32_t kVStage = 128 * 128;        // 128 keys x this CTA's 64 dims
+  static constexpr uint32_t kK = 2 * kQBox;
+  static constexpr uint32_t kV = kK + kPKStages * kKStage;
+  static constexpr uint32_t kBias = kV + kPVStages * kVStage;  // [2 parity][128] fp32
+  static constexpr uint32_t kBars = kBias + 2 * 128 * 4;
+  static constexpr uint32_t kMisc = kBars + 48 * 8;
+  static constexpr uint32_t kTotal = kMisc + 16;
+  static constexpr uint32_t kDynSmem = kTotal + 1024;
+  static_assert(kDynSmem <= 227 * 1024, "shared memory");
+};
+
+// barrier slots (same offsets in both CTAs)
+enum {
+  kPQFull = 0,     // CTA 0: Q bytes of both CTAs
+  kPQEmpty = 1,    // each CTA
+  kPSFull = 2,     // [2 buffers], each CTA
+  kPPFull = 4,     // [2 buffers], CTA 0: 256 softmax threads
+  kPOFull = 6,     // each CTA
+  kPOFree = 7,     // CTA 0: 256 softmax threads
+  kPPVDone = 8,    // each CTA, one phase per P.V
+  kPDrain = 9,     // CTA 0
+  kPKFull = 10,    // [K stages], CTA 0: both halves
+  kPKEmpty = kPKFull + kPKStages,   // [K stages], each CTA
+  kPVFull = kPKEmpty + kPKStages,   // [V stages], CTA 0
+  kPVEmpty = kPVFull + kPVStages,   // [V stages], each CTA
+  kPBarCount = kPVEmpty + kPVStages,
+};
+static_assert(kPBarCount <= 48, "barrier slots");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ TcParams p) {
+  constexpr int DH = 128;
+  constexpr bool kSplit = false;  // units are whole items (the pair plan never splits)
+  const UnitTable<false> tab{0};
+  using L = PairLay;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  float* s_bias = reinterpret_cast<float*>(smem + L::kBias);
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  auto leader_bar = [&](int i) { return mapa_shared(bar(i), 0); };
+  auto peer_bar = [&](int i) { return mapa_shared(bar(i), 1); };
+  // commit to the same barrier in both CTAs
+  auto commit_both = [&](int i) {
+    umma_commit_pair(leader_bar(i));
+    umma_commit_pair(peer_bar(i));
+  };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(bar(kPQFull), 1);
+    mbar_init(bar(kPQEmpty), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(kPSFull + b), 1);
+      mbar_init(bar(kPPFull + b), 256);
+    }
+    mbar_init(bar(kPOFull), 1);
+    mbar_init(bar(kPOFree), 256);
+    mbar_init(bar(kPPVDone), 1);
+    mbar_init(bar(kPDrain), 1);
+    for (int s = 0; s < kPKStages; ++s) {
+      mbar_init(bar(kPKFull + s), 1);
+      mbar_init(bar(kPKEmpty + s), 1);
+    }
+    for (int s = 0; s < kPVStages; ++s) {
+      mbar_init(bar(kPVFull + s), 1);
+      mbar_init(bar(kPVEmpty + s), 1);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers and TMEM of both CTAs are ready
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  int q_loads = 0, k_loads = 0, v_loads = 0;  // CTA 0's TMA thread: for the abort drain
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();  // K/V tiles are re-read by later units
+      int ks = 0, vs = 0;
+      uint32_t kph = 0, vph = 0, q_waits = 0;
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int u = snake_unit(round, cl, ncl);
+        if (u >= p.n_units) break;
+        const Unit w = decode_unit<kSplit>(p, tab, u);
+        const Item& it = w.it;
+        const int32_t kstart = p.kept_start[it.b];
+        const int head = rank ? it.hb : it.ha;
+        if (!(ok = mbar_wait(bar(kPQEmpty), (q_waits++ & 1) ^ 1, abort_flag, p.status,
+                             kDevTimeoutAttn)))
+          break;
+        if (leader) {
+          mbar_arrive_expect_tx(bar(kPQFull), 2 * 2 * L::kQBox);
+          ++q_loads;
+        }
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d_pair(sb + L::kQ + c * L::kQBox, &tm_q, head * DH + c * 64, kstart + it.t * kBM,
+                           leader_bar(kPQFull), pol);
+        for (int j = w.j0; j < w.j1; ++j) {
+          if (!(ok = mbar_wait(bar(kPKEmpty + ks), kph ^ 1, abort_flag, p.status, kDevTimeoutAttn)))
+            break;
+          if (leader) {
+            mbar_arrive_expect_tx(bar(kPKFull + ks), 2 * L::kKStage);
+            ++k_loads;
+          }
+          for (int c = 0; c < 2; ++c)
+            tma_load_2d_pair(sb + L::kK + ks * L::kKStage + c * L::kKBox, &tm_k, it.hk * DH + c * 64,
+                             kstart + j * kBN + static_cast<int>(rank) * 64, leader_bar(kPKFull + ks),
+                             pol);
+          if (++ks == kPKStages) {
+            ks = 0;
+            kph ^= 1;
+          }
+          if (!(ok = mbar_wait(bar(kPVEmpty + vs), vph ^ 1, abort_flag, p.status, kDevTimeoutAttn)))
+            break;
+          if (leader) {
+            mbar_arrive_expect_tx(bar(kPVFull + vs), 2 * L::kVStage);
+            ++v_loads;
+          }
+          tma_load_2d_pair(sb + L::kV + vs * L::kVStage, &tm_v,
+                           it.hk * DH + static_cast<int>(rank) * 64, kstart + j * kBN,
+                           leader_bar(kPVFull + vs), pol);
+          if (++vs == kPVStages) {
+            vs = 0;
+            vph ^= 1;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (CTA 0) ----------------
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(2 * kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(2 * kBM, DH, false, true);
+      uint32_t ph = 1u << kPOFree;  // bit i: parity to wait for on slot i ("free" starts passed)
+      bool ok = true;
+      auto wait_slot = [&](int slot) {
+        ok = mbar_wait(bar(slot), (ph >> slot) & 1u, abort_flag, p.status, kDevTimeoutAttn);
+        ph ^= 1u << slot;
+        return ok;
+      };
+      const uint64_t dq = sw128_desc(sb + L::kQ, 16, 1024);
+      const uint64_t dk0 = sw128_desc(sb + L::kK, 16, 1024);
+      const uint64_t dv0 = sw128_desc(sb + L::kV, L::kVStage, 1024);
+      const uint32_t t_o = tmem + 256;
+      auto issue_s = [&](int bf, int ks) {
+        const uint64_t dk = dk0 + ((ks * L::kKStage) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_ss_pair(tmem + bf * 128, dq + (kk >> 2) * (L::kQBox >> 4) + (kk & 3) * 2,
+                       dk + (kk >> 2) * (L::kKBox >> 4) + (kk & 3) * 2, idesc_qk, kk > 0 ? 1u : 0u);
+      };
+      int ks = 0, vs = 0;
+      uint32_t kph = 0, vph = 0;
+      for (int round = 0; ok; ++round) {
+        const int u = snake_unit(round, cl, ncl);
+        if (u >= p.n_units) break;
+        const Unit w = decode_unit<kSplit>(p, tab, u);
+        const int n_kv = w.j1 - w.j0;
+        if (!wait_slot(kPQFull)) break;
+        const int pro = n_kv < 2 ? n_kv : 2;
+        for (int j = 0; j < pro; ++j) {
+          if (!(ok = mbar_wait(bar(kPKFull + ks), kph, abort_flag, p.status, kDevTimeoutAttn))) break;
+          tc_fence_after();
+          issue_s(j, ks);
+          commit_both(kPSFull + j);
+          commit_both(kPKEmpty + ks);
+          if (++ks == kPKStages) {
+            ks = 0;
+            kph ^= 1;
+          }
+        }
+        if (!ok) break;
+        if (n_kv <= 2) commit_both(kPQEmpty);
+        for (int j = 0; j < n_kv; ++j) {
+          const int bf = j & 1;
+          if (!wait_slot(kPPFull + bf)) break;
+          if (j == 0 && !wait_slot(kPOFree)) break;
+          if (!(ok = mbar_wait(bar(kPVFull + vs), vph, abort_flag, p.status, kDevTimeoutAttn))) break;
+          tc_fence_after();
+          const uint64_t dv = dv0 + ((vs * L::kVStage) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ts_pair(t_o, tmem + bf * 128 + kk * 8, dv + kk * (2048 >> 4), idesc_pv,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+          commit_both(kPPVDone);
+          if (j + 1 == n_kv) commit_both(kPOFull);
+          commit_both(kPVEmpty + vs);
+          if (++vs == kPVStages) {
+            vs = 0;
+            vph ^= 1;
+          }
+          if (j + 2 < n_kv) {
+            if (!(ok = mbar_wait(bar(kPKFull + ks), kph, abort_flag, p.status, kDevTimeoutAttn)))
+              break;
+            tc_fence_after();
+            issue_s(bf, ks);  // P(j) in this buffer was read by the P.V above: in order
+            commit_both(kPSFull + bf);
+            commit_both(kPKEmpty + ks);
+            if (++ks == kPKStages) {
+              ks = 0;
+              kph ^= 1;
+            }
+            if (j + 3 == n_kv) commit_both(kPQEmpty);  // that was the unit's last S
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax (warps 2-5, this CTA's head) ----------------
+    const int x = static_cast<int>(rank);  // head slot within the pair
+    const int quarter = warp & 3;
+    const int rl = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off;
+    const uint32_t t_o = tmem + lane_off + 256;
+    uint32_t s_ph = 0, o_waits = 0, tile_ctr = 0;
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      const int u = snake_unit(round, cl, ncl);
+      if (u >= p.n_units) break;
+      const Unit w = decode_unit<kSplit>(p, tab, u);
+      const Item& it = w.it;
+      const int head = x ? it.hb : it.ha;
+      const int32_t kstart = p.kept_start[it.b];
+      const int32_t len = p.kept_start[it.b + 1] - kstart;
+      const int n_kv = w.j1 - w.j0;
+      const float scale = kLog2e / (sqrtf(static_cast<float>(DH)) * __ldg(p.temp + head));
+      const float gl = __ldg(p.gain + head) * kLog2e;
+      const float2 sc2 = make_float2(scale, scale);
+      float m = -INFINITY, l = 0.0f;
+      const int key0 = w.j0 * kBN + rl;
+      float next_bias = (p.logsig && key0 < len) ? gl * __ldg(p.logsig + kstart + key0) : 0.0f;
+      for (int j = 0; j < n_kv; ++j) {
+        const int jabs = w.j0 + j;
+        const int bf = j & 1;
+        float* bias = s_bias + (tile_ctr & 1) * 128;
+        bias[rl] = next_bias;
+        if (j + 1 < n_kv) {
+          const int key = (jabs + 1) * kBN + rl;
+          next_bias = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
+        }
+        ok = mbar_wait(bar(kPSFull + bf), (s_ph >> bf) & 1u, abort_flag, p.status, kDevTimeoutAttn);
+        s_ph ^= 1u << bf;
+        if (named_barrier_or(1, 128, !ok)) {  // one outcome for the warpgroup; bias visible
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + bf * 128 + c * 32, sr[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+        float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const float4* b4 = reinterpret_cast<const float4*>(bias);
+        if (jabs != it.t) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 bb = b4[(c * 32 + e) >> 2];
+              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
+                                     sc2, make_float2(bb.x, bb.y));
+              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
+                                     sc2, make_float2(bb.z, bb.w));
+              sr[c][e] = __float_as_uint(t0.x);
+              sr[c][e + 1] = __float_as_uint(t0.y);
+              sr[c][e + 2] = __float_as_uint(t1.x);
+              sr[c][e + 3] = __float_as_uint(t1.y);
+              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
+              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
+            }
+          }
+        } else {  // diagonal tile: key column c is visible to row rl iff c <= rl
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const int col = c * 32 + e;
+              const float4 bb = b4[col >> 2];
+              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
+                                     sc2, make_float2(bb.x, bb.y));
+              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
+                                     sc2, make_float2(bb.z, bb.w));
+              if (col > rl) t0.x = -INFINITY;
+              if (col + 1 > rl) t0.y = -INFINITY;
+              if (col + 2 > rl) t1.x = -INFINITY;
+              if (col + 3 > rl) t1.y = -INFINITY;
+              sr[c][e] = __float_as_uint(t0.x);
+              sr[c][e + 1] = __float_as_uint(t0.y);
+              sr[c][e + 2] = __float_as_uint(t1.x);
+              sr[c][e + 3] = __float_as_uint(t1.y);
+              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
+              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
+            }
+          }
+        }
+        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+        float alpha = 1.0f;
+        const bool grow = mx > m + kRescaleLog2;
+        if (grow) {
+          alpha = exp2_approx(m - mx);
+          m = mx;
+        }
+        // O holds this unit's earlier P.V; rescaling it needs the last one done
+        // (warp-uniform: tcgen05.ld/st are collective)
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          if (!mbar_wait(bar(kPPVDone), (tile_ctr - 1) & 1, abort_flag, p.status, kDevTimeoutAttn))
+            ok = false;
+          tc_fence_after();
+          if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+              uint32_t orow[32];
+              tmem_ld32(t_o + c * 32, orow);
+              tmem_ld_wait(orow);
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float2 v2 = __fmul2_rn(
+                    make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
+                    make_float2(alpha, alpha));
+                orow[e] = __float_as_uint(v2.x);
+                orow[e + 1] = __float_as_uint(v2.y);
+              }
+              tmem_st32(t_o + c * 32, orow);
+            }
+          }
+        }
+        ++tile_ctr;
+        const float2 nm2 = make_float2(-m, -m);
+        float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 a2 = __fadd2_rn(
+                make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), nm2);
+            const float2 p2 = make_float2(exp2_approx(a2.x), exp2_approx(a2.y));
+            acc[(e >> 1) & 1] = __fadd2_rn(acc[(e >> 1) & 1], p2);
+            __nv_bfloat162 pp = __floats2bfloat162_rn(p2.x, p2.y);
+            pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
+          }
+          tmem_st16(t_s + bf * 128 + c * 16, pk);
+        }
+        l = fmaf(l, alpha, (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive_cluster(leader_bar(kPPFull + bf));
+      }
+      if (named_barrier_or(1, 128, !ok)) {  // a rescale wait may have failed on the last tile
+        ok = false;
+        break;
+      }
+      ok = mbar_wait(bar(kPOFull), o_waits++ & 1, abort_flag, p.status, kDevTimeoutAttn);
+      if (named_barrier_or(1, 128, !ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int qi = it.t * kBM + rl;
+      const float inv = 1.0f / l;
+      __nv_bfloat16* out = p.out + (static_cast<int64_t>(kstart + qi) * p.hq + head) * DH;
+#pragma unroll
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t orow[32];
+        tmem_ld32(t_o + c * 32, orow);
+        tmem_ld_wait(orow);
+        if (qi < len) {
+          uint32_t pkd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(orow[2 * e]) * inv,
+                                                      __uint_as_float(orow[2 * e + 1]) * inv);
+            pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(leader_bar(kPOFree));
+      if (p.lse && qi < len)
+        p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (m + log2f(l)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && leader) {
+    // a wait gave up: let the loads (both CTAs' bytes land on these barriers)
+    // and the MMAs already issued finish (bounded) before memory is released
+    if (warp == 0 && lane == 0) {
+      if (q_loads > 0) mbar_drain(bar(kPQFull), (q_loads - 1) & 1);
+      for (int s = 0; s < kPKStages && s < k_loads; ++s)
+        mbar_drain(bar(kPKFull + s), ((k_loads - 1 - s) / kPKStages) & 1);
+      for (int s = 0; s < kPVStages && s < v_loads; ++s)
+        mbar_drain(bar(kPVFull + s), ((v_loads - 1 - s) / kPVStages) & 1);
+    }
+    if (warp == 1 && lane == 0) {
+      umma_commit_pair(leader_bar(kPDrain));
+      mbar_drain(bar(kPDrain), 0);
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();  // no commit, arrival or load can still target the other CTA
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host: work plan.  Items are enumerated in the kernel's rank order (query-tile
 // level descending, prompts longest first, head pairs); an item at level t has
 // t + 1 key tiles.  For k = 1..kMaxChunks chunks of the longest item, items
 // longer than C = ceil(max / k) tiles are cut into ceil(n / C) chunks; the plan
 // with the smallest modelled makespan under the kernel's boustrophedon deal
-// wins (a split must gain at least 3 % to be taken).  Cost model, in key
-// tiles: a unit costs its tiles plus 0.3 (Q load, epilogue), a chunk of a
-// split item 1.0 more (partial store and merge).
+// wins (a split must gain at least 3 % to be taken).  Cost model, in times of
+// one key tile of a head pair on one SM (measured): a unit costs its tiles
+// plus 0.5 (Q load, epilogue), a chunk of a split item 3 more (partial store
+// and merge).  The pair kernel runs a tile in 0.72 of that, but on two SMs.
 // ---------------------------------------------------------------------------
 struct AttnPlan {
+  double span = 0.0;  // modelled makespan (0: not modelled)
   int grid = 0;
   int n_units = 0;
   int n_slots = 0;
@@ -718,12 +1183,12 @@ static double snake_makespan(const double* cost_sorted, int n, int g, double* lo
 
 // Fills `tab` (when non-null and the plan splits) and returns the plan.
 static AttnPlan make_plan(const TcParams& p, int dh, int n_sms, bool allow_split,
-                          UnitTable<true>* tab) {
-  constexpr double kOverhead = 0.3, kChunkCost = 1.0;
+                          UnitTable<true>* tab, double kTile, double kChunkCost) {
+  constexpr double kOverhead = 0.5;
   AttnPlan best;
   best.n_units = p.n_items;
   best.grid = p.n_items < n_sms ? p.n_items : n_sms;
-  if (!allow_split || p.n_items > kMaxUnits || p.n_items == 0) return best;
+  if (p.n_items > kMaxUnits || p.n_items == 0) return best;
   const int n = p.n_items;
   int32_t nkv[kMaxUnits];
   item_lengths(p, nkv);
@@ -738,7 +1203,7 @@ static AttnPlan make_plan(const TcParams& p, int dh, int n_sms, bool allow_split
   const int g_cap = n_sms < 1024 ? n_sms : 1024;
   double base = 0.0;
   double best_span = 0.0;
-  for (int k = 1; k <= kMaxChunks; ++k) {
+  for (int k = 1; k <= (allow_split ? kMaxChunks : 1); ++k) {
     const int C = (max_n + k - 1) / k;
     if (k > 1 && C == (max_n + k - 2) / (k - 1)) continue;
     int nu = 0;
@@ -751,7 +1216,7 @@ static AttnPlan make_plan(const TcParams& p, int dh, int n_sms, bool allow_split
       }
       for (int c = 0; c < s; ++c) {
         const int lo = c * nkv[i] / s, hi = (c + 1) * nkv[i] / s;
-        units[nu++] = {hi - lo + kOverhead + (s > 1 ? kChunkCost : 0.0), i, c, s};
+        units[nu++] = {kTile * (hi - lo) + kOverhead + (s > 1 ? kChunkCost : 0.0), i, c, s};
       }
     }
     if (!fits) continue;
@@ -801,6 +1266,7 @@ static AttnPlan make_plan(const TcParams& p, int dh, int n_sms, bool allow_split
       }
     }
   }
+  best.span = best_span;
   if (best.split) best.workspace = split_workspace_bytes(best.n_slots, dh);
   return best;
 }
@@ -864,12 +1330,59 @@ tg_status launch_dh(const void* q, const void* k, const void* v, const TcParams&
   return cuda_check(cudaGetLastError(), "attn_tc launch");
 }
 
+tg_status launch_pair(const void* q, const void* k, const void* v, const TcParams& p, int clusters,
+                      int hkv, cudaStream_t st) {
+  constexpr int DH = 128;
+  CUtensorMap tq, tk, tv;
+  const uint64_t M = static_cast<uint64_t>(p.m_total);
+  if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(p.hq) * DH, M,
+                           static_cast<uint64_t>(p.hq) * DH * 2, 64, kBM) ||
+      !encode_tmap_2d_bf16(&tk, k, static_cast<uint64_t>(hkv) * DH, M,
+                           static_cast<uint64_t>(hkv) * DH * 2, 64, 64) ||
+      !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(hkv) * DH, M,
+                           static_cast<uint64_t>(hkv) * DH * 2, 64, kBN))
+    return set_error(TG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q/k/v");
+  tg_status r = cuda_check(cudaFuncSetAttribute(attn_pair_kernel,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(PairLay::kDynSmem)),
+                           "attn pair smem attribute");
+  if (r != TG_OK) return r;
+  attn_pair_kernel<<<2 * clusters, kPairThreads, PairLay::kDynSmem, st>>>(tq, tk, tv, p);
+  return cuda_check(cudaGetLastError(), "attn_pair launch");
+}
+
+// CTA pairs need an even group (both heads of every pair exist) and head_dim 128.
+// They can pay off only for small batches, whose items cannot fill one SM
+// each (a unit then runs on two SMs); the single-CTA kernel, two softmax
+// warpgroups per SM, has the higher throughput per SM.  The modelled
+// makespans of the two plans decide.
+constexpr double kTilePair = 0.72;  // pair kernel's tile time, in single-CTA tile times
+constexpr double kMergeCost = 3.0;
+static bool pairs_possible(const TcParams& p, int hkv, int dh) {
+  return dh == 128 && (p.hq / hkv) % 2 == 0 && num_sms() >= 2 && p.n_items <= num_sms();
+}
+static AttnPlan choose_plan(const TcParams& p, int hkv, int dh, bool allow_split,
+                            UnitTable<true>* tab_single, bool* pairs) {
+  AttnPlan plan = make_plan(p, dh, num_sms(), allow_split, tab_single, 1.0, kMergeCost);
+  *pairs = false;
+  if (pairs_possible(p, hkv, dh)) {
+    // whole items only: with two SMs per unit, splitting does not pay for its merges
+    const AttnPlan pp = make_plan(p, dh, num_sms() / 2, false, nullptr, kTilePair, kMergeCost);
+    if (pp.span > 0.0 && pp.span < plan.span) {
+      plan = pp;
+      *pairs = true;
+    }
+  }
+  return plan;
+}
+
 }  // namespace
 
 size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh) {
   TcParams p;
   if (fill_params(pt, hq, hkv, &p) != TG_OK || p.n_items == 0) return 0;
-  return make_plan(p, dh, num_sms(), true, nullptr).workspace;
+  bool pairs = false;
+  return choose_plan(p, hkv, dh, true, nullptr, &pairs).workspace;
 }
 
 tg_status launch_attn_tc(const void* q, const void* k, const void* v, const PromptTable& pt,
@@ -886,8 +1399,9 @@ tg_status launch_attn_tc(const void* q, const void* k, const void* v, const Prom
   p.temp = temp;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  static thread_local UnitTable<true> tab;
-  const AttnPlan plan = make_plan(p, dh, num_sms(), workspace != nullptr, &tab);
+  static thread_local UnitTable<true> tab;  // split plans are single-CTA plans
+  bool pairs = false;
+  const AttnPlan plan = choose_plan(p, hkv, dh, workspace != nullptr, &tab, &pairs);
   if (plan.split && workspace_bytes < plan.workspace)
     return set_error(TG_ERR_WORKSPACE, "attention workspace: %zu bytes given, %zu needed",
                      workspace_bytes, plan.workspace);
@@ -895,6 +1409,7 @@ tg_status launch_attn_tc(const void* q, const void* k, const void* v, const Prom
   if (!p.status) return set_error(TG_ERR_CUDA, "device status word unavailable");
   if (!plan.split) {
     const UnitTable<false> none{0};
+    if (pairs) return launch_pair(q, k, v, p, plan.grid, hkv, st);
     if (dh == 64) return launch_dh<64, false>(q, k, v, p, none, plan.grid, hkv, st);
     return launch_dh<128, false>(q, k, v, p, none, plan.grid, hkv, st);
   }

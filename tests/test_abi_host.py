@@ -173,7 +173,7 @@ def test_attention_workspace_plan(L):
 
     if torch.cuda.is_available():
         pytest.skip("plan sizes below assume 148 SMs")
-    st, b = _ws_bytes(L, [0, 2304])  # one 16k-token prompt kept down to 2304 rows
+    st, b = _ws_bytes(L, [0, 1280])  # one 32k-token prompt kept down to 1280 rows
     assert st == 0 and b > 0
     # every partial slot holds 2 heads x 128 rows x (head_dim + 1) floats, plus counters
     assert b % 4 == 0 and b >= 2 * 128 * 129 * 4
@@ -187,8 +187,8 @@ def test_attention_workspace_plan(L):
     _, ck = _arr([0, 10])
     assert L.tg_attention_workspace_bytes(0, 1, ck, 16, 8, 128, 0, None) == INVALID
     # a workspace smaller than the plan needs is refused before anything launches
-    st, need = _ws_bytes(L, [0, 2304])
-    _, ck = _arr([0, 2304])
+    st, need = _ws_bytes(L, [0, 1280])
+    _, ck = _arr([0, 1280])
     a = L.tg_gated_attention
     assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, FAKE,
              need - 16, 0, None) == WORKSPACE
