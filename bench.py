@@ -421,6 +421,103 @@ def run_ncu_case(args):
                       "M": layer.M}))
 
 
+def run_extras(args):
+    """Supplementary layer-level figures for one workload (one JSON line; not the
+    bench line): the bias overhead of the gated attention (logsig vs none), the
+    ungated full-N causal attention over every token of the same prompts, the
+    gated step's stages for comparison, and the live device memory of one gated
+    layer vs a full-N layer."""
+    import torch
+
+    import learned_token_pruning_gate_b200 as tg
+    from learned_token_pruning_gate_b200 import inputs as gen
+    from learned_token_pruning_gate_b200.pipeline import GatedLayer
+
+    w = gen.WORKLOADS[args.workload]
+    inp = gen.make_inputs(w)
+    dev = torch.device("cuda", 0)
+    d = lambda t: t.to(dev).contiguous()  # noqa: E731
+    res = [d(x) for x in (inp.h, inp.q, inp.k, inp.v, inp.W1, inp.b1, inp.w2, inp.gain, inp.temp)]
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated()  # inputs resident: count what the step allocates
+    torch.cuda.reset_peak_memory_stats()
+    layer = GatedLayer(*res[:7], inp.b2, res[7], res[8], inp.cu_seqlens, inp.doc_begin,
+                       inp.doc_end, inp.budget, rope_theta=w.rope_theta, algo=tg.ALGO_AUTO)
+    layer.run()
+    torch.cuda.synchronize()
+    gated_peak = torch.cuda.max_memory_allocated() - base
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(HOLD_CYCLES // 4)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return float(np.median(ms)) * 1e3  # us
+
+    import ctypes
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    stage_us = {s: timed(lambda s=s: getattr(layer, s)(st), 20) for s in GatedLayer.STAGES}
+    ws = layer.workspace
+    with_bias = timed(lambda: tg.gated_attention(layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host,
+                                                 layer.logsig, layer.gain, layer.temp,
+                                                 out=layer.out, workspace=ws), 20)
+    no_bias = timed(lambda: tg.gated_attention(layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host,
+                                               None, layer.gain, layer.temp, out=layer.out,
+                                               workspace=ws), 20)
+    del layer
+    torch.cuda.synchronize()
+    # ungated: every token of every prompt attends causally, no bias (the layer without a gate)
+    q, k, v = res[1], res[2], res[3]
+    base = torch.cuda.memory_allocated()
+    torch.cuda.reset_peak_memory_stats()
+    out = torch.empty_like(q)
+    lens = np.diff(np.asarray(inp.cu_seqlens))
+    full_ws = tg.attention_workspace_bytes(inp.cu_seqlens, w.n_q_heads, w.n_kv_heads, w.head_dim)
+    fws = torch.empty(full_ws, dtype=torch.uint8, device=dev) if full_ws else None
+    gain, temp = res[7], res[8]
+    reps = 3 if w.total_tokens > 40000 else 10
+    ungated = timed(lambda: tg.gated_attention(q, k, v, inp.cu_seqlens, None, gain, temp, out=out,
+                                               workspace=fws), reps)
+    torch.cuda.synchronize()
+    full_peak = torch.cuda.max_memory_allocated() - base
+    hq, dh = w.n_q_heads, w.head_dim
+    esz = 2 if w.dtype == "bf16" else 4
+    full_flops = float(sum(2.0 * dh * hq * n * (n + 1) for n in lens))
+    gated_total = sum(stage_us.values())
+    print(json.dumps({
+        "extras": args.workload, "tokens": w.total_tokens, "kept": w.kept_lengths(),
+        "stage_us": {s: round(v, 2) for s, v in stage_us.items()},
+        "gated_layer_us": round(gated_total, 2),
+        "bias_overhead": {"with_bias_us": round(with_bias, 2), "no_bias_us": round(no_bias, 2),
+                          "ratio": round(with_bias / no_bias, 4)},
+        "ungated_attention": {"us": round(ungated, 2), "tflops": round(full_flops / ungated / 1e6, 1),
+                              "frac_measured_bf16": round(full_flops / ungated / 1e6 / _peaks()["bf16"], 4)},
+        "speedup_vs_ungated_attention": round(ungated / gated_total, 2),
+        "memory_bytes": {
+            "gated_step_allocated": int(gated_peak), "ungated_step_allocated": int(full_peak),
+            "kv_gated": int(2 * sum(w.kept_lengths()) * w.n_kv_heads * dh * esz),
+            "kv_ungated": int(2 * w.total_tokens * w.n_kv_heads * dh * esz),
+            "attention_live_gated": int(sum(w.kept_lengths()) * (2 * hq + 2 * w.n_kv_heads) * dh * esz),
+            "attention_live_ungated": int(w.total_tokens * (2 * hq + 2 * w.n_kv_heads) * dh * esz)},
+        "note": "one layer: ungated = causal attention over all N tokens (q,k,v already resident); "
+                "gated = gate + top-K + compaction + gated attention; *_step_allocated = device "
+                "memory each step allocates with its inputs resident (gated: z, kept rows, "
+                "compacted h/q/k/v, bias, output, workspace; ungated: output); kv_* and "
+                "attention_live_* (q, k, v, o) are the tensor sizes the layer holds",
+    }), flush=True)
+
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,11 +527,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extras", action="store_true",
+                    help="print bias overhead, ungated full-N attention and memory figures")
     ap.add_argument("--ncu-case", action="store_true",
                     help="untimed: run --steps plain steps of the workload (profiling)")
     args = ap.parse_args()
     if args.ncu_case:
         run_ncu_case(args)
+    elif args.extras:
+        run_extras(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
