@@ -212,6 +212,23 @@ TG_API tg_status tg_attention_workspace_bytes(tg_dtype dtype, int32_t batch, con
                                        int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                        int32_t algo, size_t* bytes_out);
 
+/* The attention kernels tg_gated_attention chooses between. */
+typedef enum {
+    TG_ATTN_SIMT = 0,      /* CUDA-core kernel */
+    TG_ATTN_TC = 1,        /* tcgen05 kernel, one SM per (query tile, head pair) */
+    TG_ATTN_TC_SPLIT = 2,  /* same, long query tiles split by key range (uses the workspace) */
+    TG_ATTN_TC_PAIR = 3    /* tcgen05 kernel on CTA pairs, two SMs per (query tile, head pair) */
+} tg_attn_kernel;
+
+/*
+ * Which kernel tg_gated_attention launches for this batch and head shape on
+ * the current device (a tg_attn_kernel in *kernel_out).  with_workspace: the
+ * call will receive a workspace of tg_attention_workspace_bytes.  Host-only.
+ */
+TG_API tg_status tg_attention_kernel(tg_dtype dtype, int32_t batch, const int32_t* cu_kept_h,
+                              int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                              int32_t algo, int32_t with_workspace, int32_t* kernel_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,7 @@ __all__ = [
     "TG_BF16", "TG_FP32", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "TokenGateError",
     "library", "kept_offsets", "gate_score", "topk_select", "compact_gather", "gated_attention",
     "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
+    "attention_kernel",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -37,8 +38,10 @@ LIB_PATH = os.path.join(_HERE, "libtokengate.so")
 EXPORTED_SYMBOLS = (
     "tg_status_string", "tg_last_error_message", "tg_version", "tg_device_status",
     "tg_kept_offsets", "tg_gate_score", "tg_topk_select", "tg_compact_gather",
-    "tg_gated_attention", "tg_attention_workspace_bytes",
+    "tg_gated_attention", "tg_attention_workspace_bytes", "tg_attention_kernel",
 )
+ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
+                3: "attn_pair_kernel"}
 
 
 class TokenGateError(RuntimeError):
@@ -84,6 +87,8 @@ def library():
                                      _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _i32, _vp]
     L.tg_attention_workspace_bytes.argtypes = [ctypes.c_int, _i32, _i32p, _i32, _i32, _i32, _i32,
                                                ctypes.POINTER(ctypes.c_size_t)]
+    L.tg_attention_kernel.argtypes = [ctypes.c_int, _i32, _i32p, _i32, _i32, _i32, _i32, _i32,
+                                      ctypes.POINTER(ctypes.c_int32)]
     for name in EXPORTED_SYMBOLS:
         if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -231,6 +236,18 @@ def attention_workspace_bytes(cu_kept_host, n_q_heads, n_kv_heads, head_dim, dty
     _check("tg_attention_workspace_bytes", library().tg_attention_workspace_bytes(
         code, len(cu) - 1, cu_p, n_q_heads, n_kv_heads, head_dim, algo, ctypes.byref(out)))
     return int(out.value)
+
+
+def attention_kernel(cu_kept_host, n_q_heads, n_kv_heads, head_dim, dtype="bf16",
+                     algo=ALGO_AUTO, with_workspace=True):
+    """Name of the attention kernel tg_gated_attention launches for this batch."""
+    cu, cu_p = _host_i32(cu_kept_host)
+    code = 0 if dtype in ("bf16", torch.bfloat16) else 1
+    out = ctypes.c_int32(-1)
+    _check("tg_attention_kernel", library().tg_attention_kernel(
+        code, len(cu) - 1, cu_p, n_q_heads, n_kv_heads, head_dim, algo, int(with_workspace),
+        ctypes.byref(out)))
+    return ATTN_KERNELS[out.value]
 
 
 def gated_attention(q, k, v, cu_kept_host, logsig=None, gain=None, temp=None, out=None,

@@ -318,6 +318,26 @@ tg_status tg_attention_workspace_bytes(tg_dtype dtype, int32_t batch, const int3
   return TG_OK;
 }
 
+tg_status tg_attention_kernel(tg_dtype dtype, int32_t batch, const int32_t* cu_kept_h,
+                              int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                              int32_t algo, int32_t with_workspace, int32_t* kernel_out) {
+  if (!kernel_out) return set_error(TG_ERR_INVALID_ARG, "kernel_out is null");
+  size_t bytes = 0;
+  tg_status r = tg_attention_workspace_bytes(dtype, batch, cu_kept_h, n_q_heads, n_kv_heads,
+                                             head_dim, algo, &bytes);  // validates the arguments
+  if (r != TG_OK) return r;
+  if (dtype != TG_BF16 || algo == TG_ALGO_SIMT) {
+    *kernel_out = TG_ATTN_SIMT;
+    return TG_OK;
+  }
+  PromptTable t;
+  int max_len = 0;
+  r = build_kept_table(batch, cu_kept_h, &t, &max_len);
+  if (r != TG_OK) return r;
+  *kernel_out = attn_tc_kernel_choice(t, n_q_heads, n_kv_heads, head_dim, with_workspace != 0);
+  return TG_OK;
+}
+
 tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dtype dtype,
                              int32_t batch, const int32_t* cu_kept_h, int32_t n_q_heads,
                              int32_t n_kv_heads, int32_t head_dim, const float* logsig,

@@ -1378,6 +1378,14 @@ static AttnPlan choose_plan(const TcParams& p, int hkv, int dh, bool allow_split
 
 }  // namespace
 
+int attn_tc_kernel_choice(const PromptTable& pt, int hq, int hkv, int dh, bool with_workspace) {
+  TcParams p;
+  if (fill_params(pt, hq, hkv, &p) != TG_OK || p.n_items == 0) return TG_ATTN_TC;
+  bool pairs = false;
+  const AttnPlan plan = choose_plan(p, hkv, dh, with_workspace, nullptr, &pairs);
+  return pairs ? TG_ATTN_TC_PAIR : plan.split ? TG_ATTN_TC_SPLIT : TG_ATTN_TC;
+}
+
 size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh) {
   TcParams p;
   if (fill_params(pt, hq, hkv, &p) != TG_OK || p.n_items == 0) return 0;

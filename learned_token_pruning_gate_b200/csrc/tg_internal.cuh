@@ -61,6 +61,8 @@ tg_status launch_attn_tc(const void* q, const void* k, const void* v, const Prom
                          void* workspace, size_t workspace_bytes, cudaStream_t st);
 // Workspace the tensor-core attention uses to split long items on this device (0 = none).
 size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh);
+// The tg_attn_kernel the tensor-core attention launches for this batch.
+int attn_tc_kernel_choice(const PromptTable& pt, int hq, int hkv, int dh, bool with_workspace);
 
 // Tensor map encoding through the driver entry point (no libcuda link).
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,

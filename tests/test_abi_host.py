@@ -195,6 +195,22 @@ def test_attention_workspace_plan(L):
     assert b"needed" in L.tg_last_error_message()
 
 
+def test_attention_kernel_choice():
+    """The per-call plan on 148 SMs: CTA pairs when a small batch cannot fill the
+    GPU, key-range split when that balances better, one SM per unit otherwise."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("choices below assume 148 SMs")
+    assert tg.attention_kernel([0, 2304], 16, 8, 128) == "attn_pair_kernel"
+    assert tg.attention_kernel([0, 1280], 16, 8, 128) == "attn_tc_kernel (key-range split)"
+    assert tg.attention_kernel([0, 1280], 16, 8, 128, with_workspace=False) == "attn_pair_kernel"
+    assert tg.attention_kernel([0, 8448], 16, 8, 128) == "attn_tc_kernel"
+    assert tg.attention_kernel([0, 2304], 12, 4, 128, with_workspace=False) == "attn_tc_kernel"
+    assert tg.attention_kernel([0, 2304], 16, 8, 64, with_workspace=False) == "attn_tc_kernel"
+    assert tg.attention_kernel([0, 2304], 16, 8, 128, dtype="fp32") == "attn_simt_kernel"
+
+
 def test_no_gpu_means_cuda_error_not_crash(L):
     import torch
 
