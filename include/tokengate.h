@@ -229,6 +229,28 @@ TG_API tg_status tg_attention_kernel(tg_dtype dtype, int32_t batch, const int32_
                               int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                               int32_t algo, int32_t with_workspace, int32_t* kernel_out);
 
+/*
+ * tg_gated_attention for callers that cannot allocate device memory (the
+ * pages have no counterpart: this is a deployment convenience).  A serving
+ * process whose allocator reserved the whole GPU up front, or code that must
+ * not allocate around CUDA-graph capture, cannot provide the attention
+ * workspace; this call takes the scratch from a fixed array built into the
+ * library instead: 32 MiB of device memory, held by every GPU that loads the
+ * library until the process exits.
+ *   Arguments, results and errors are those of tg_gated_attention without the
+ *   workspace.  A batch whose split plan needs more scratch than the array
+ *   holds returns TG_ERR_WORKSPACE before anything launches.
+ *   The first call on a device looks up the array's address (a runtime call,
+ *   no allocation): make it before any stream capture on that device.
+ *   All calls share the array: calls that run on the GPU at the same time race
+ *   on it, so issue them in order on one stream.  The call allocates nothing.
+ */
+TG_API tg_status tg_gated_attention_noalloc(const void* q, const void* k, const void* v, tg_dtype dtype,
+                                     int32_t batch, const int32_t* cu_kept_h, int32_t n_q_heads,
+                                     int32_t n_kv_heads, int32_t head_dim, const float* logsig,
+                                     const float* gain, const float* temp, void* out, float* lse,
+                                     int32_t algo, tg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

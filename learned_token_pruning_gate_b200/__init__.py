@@ -39,6 +39,7 @@ EXPORTED_SYMBOLS = (
     "tg_status_string", "tg_last_error_message", "tg_version", "tg_device_status",
     "tg_kept_offsets", "tg_gate_score", "tg_topk_select", "tg_compact_gather",
     "tg_gated_attention", "tg_attention_workspace_bytes", "tg_attention_kernel",
+    "tg_gated_attention_noalloc",
 )
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
                 3: "attn_pair_kernel"}
@@ -89,6 +90,8 @@ def library():
                                                ctypes.POINTER(ctypes.c_size_t)]
     L.tg_attention_kernel.argtypes = [ctypes.c_int, _i32, _i32p, _i32, _i32, _i32, _i32, _i32,
                                       ctypes.POINTER(ctypes.c_int32)]
+    L.tg_gated_attention_noalloc.argtypes = [_vp, _vp, _vp, ctypes.c_int, _i32, _i32p, _i32, _i32,
+                                             _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
     for name in EXPORTED_SYMBOLS:
         if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
             getattr(L, name).restype = ctypes.c_int

@@ -1,0 +1,74 @@
+// Gated attention without any device allocation by the caller.
+//
+// tg_gated_attention can split the key range of long query tiles when the batch
+// is too small to fill the GPU, and then needs scratch memory for the partial
+// results; normally the caller passes it as a workspace.  Some callers cannot
+// allocate device memory at all: a serving process whose allocator reserved the
+// whole device up front (so a new cudaMalloc would fail or fragment its pool),
+// or a host that must not allocate between the setup of a CUDA graph and its
+// capture.  For them tg_gated_attention_noalloc takes its scratch from one
+// fixed array compiled into the library.
+//
+// The array lives in device memory of every GPU whose context loads the
+// library, until the process exits (kScratchBytes per GPU).  Its device address
+// is looked up once per device, on that device's first call (make the first
+// call before any stream capture).  All calls share the array, so two calls
+// that run on the GPU at the same time -- on different streams, or from
+// different threads -- race on it; order them on one stream.  Each call clears
+// the array's arrival counters on its stream before the kernel runs (the
+// attention launch does this for any workspace), nothing else must start at
+// zero.
+#include <mutex>
+
+#include "tg_internal.cuh"
+
+namespace tg {
+namespace {
+
+constexpr size_t kScratchBytes = size_t(32) << 20;  // 32 MiB
+
+static __device__ __align__(256) uint8_t g_attn_scratch[kScratchBytes];
+
+// Device address of the array for the current device (nullptr on failure).
+void* scratch_address() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+}  // namespace tg
+
+using namespace tg;
+
+extern "C" {
+
+tg_status tg_gated_attention_noalloc(const void* q, const void* k, const void* v, tg_dtype dtype,
+                                     int32_t batch, const int32_t* cu_kept_h, int32_t n_q_heads,
+                                     int32_t n_kv_heads, int32_t head_dim, const float* logsig,
+                                     const float* gain, const float* temp, void* out, float* lse,
+                                     int32_t algo, tg_stream_t stream) {
+  size_t need = 0;
+  tg_status r = tg_attention_workspace_bytes(dtype, batch, cu_kept_h, n_q_heads, n_kv_heads,
+                                             head_dim, algo, &need);
+  if (r != TG_OK) return r;
+  if (need > kScratchBytes)
+    return set_error(TG_ERR_WORKSPACE,
+                     "this batch needs %zu bytes of attention scratch; the built-in array of "
+                     "tg_gated_attention_noalloc holds %zu (use tg_gated_attention with a workspace)",
+                     need, kScratchBytes);
+  void* scratch = scratch_address();
+  if (!scratch) return set_error(TG_ERR_CUDA, "cannot resolve the attention scratch array");
+  return tg_gated_attention(q, k, v, dtype, batch, cu_kept_h, n_q_heads, n_kv_heads, head_dim,
+                            logsig, gain, temp, out, lse, scratch, kScratchBytes, algo, stream);
+}
+
+}  // extern "C"
