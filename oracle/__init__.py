@@ -51,6 +51,8 @@ def _load():
                                      ctypes.c_int64, _f64p]
         L.tgo_topk_select.argtypes = [_f32p, ctypes.c_int32, _i32p, _i32p, _i32p, _i32p,
                                       _i32p, _i32p]
+        L.tgo_select_by_keys.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32, _i32p,
+                                         _i32p, _i32p, _i32p, _i32p, _i32p]
         L.tgo_gather_rows.argtypes = [_i32p, ctypes.c_int64, ctypes.c_int32, _i32p, _f32p,
                                       ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                       ctypes.c_double, _f64p]
@@ -60,8 +62,8 @@ def _load():
                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                           _f32p, _f32p, _f32p, _i64p, ctypes.c_int64, _f64p,
                                           _f64p]
-        for name in ("tgo_gate_score", "tgo_topk_select", "tgo_gather_rows", "tgo_logsig",
-                     "tgo_gated_attention"):
+        for name in ("tgo_gate_score", "tgo_topk_select", "tgo_select_by_keys",
+                     "tgo_gather_rows", "tgo_logsig", "tgo_gated_attention"):
             getattr(L, name).restype = ctypes.c_int
     return _lib
 
@@ -122,6 +124,27 @@ def topk_select(z, cu_seqlens, doc_begin, doc_end, budget):
     cu_kept = np.empty(B + 1, np.int32)
     _check(L.tgo_topk_select(_p(z, _f32p), B, _p(cu, _i32p), _p(s, _i32p), _p(e, _i32p),
                              _p(k, _i32p), _p(kept, _i32p), _p(cu_kept, _i32p)), "topk_select")
+    return kept[: int(cu_kept[-1])].copy(), cu_kept
+
+
+def select_by_keys(keys, cu_seqlens, doc_begin, doc_end, budget):
+    """Random-K selection: per prompt, the K document tokens with the largest
+    caller-drawn uint32 keys (lower index on ties), question protected.
+
+    Returns (kept_idx [M] int32 global rows ascending per prompt, cu_kept [B+1]).
+    """
+    L = _load()
+    keys = np.ascontiguousarray(keys, np.uint32)
+    cu = _c(cu_seqlens, np.int32)
+    s = _c(doc_begin, np.int32)
+    e = _c(doc_end, np.int32)
+    k = _c(budget, np.int32)
+    B = s.shape[0]
+    kept = np.empty(max(int(cu[-1]), 1), np.int32)
+    cu_kept = np.empty(B + 1, np.int32)
+    _check(L.tgo_select_by_keys(keys.ctypes.data_as(ctypes.POINTER(ctypes.c_uint32)), B,
+                                _p(cu, _i32p), _p(s, _i32p), _p(e, _i32p), _p(k, _i32p),
+                                _p(kept, _i32p), _p(cu_kept, _i32p)), "select_by_keys")
     return kept[: int(cu_kept[-1])].copy(), cu_kept
 
 

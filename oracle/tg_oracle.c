@@ -18,6 +18,7 @@
  *      residual                                   -> tgo_gate_score
  *   2. A top-K selector keeps the K highest-scoring document tokens; question
  *      tokens are never pruned                    -> tgo_topk_select
+ *      (random-K ablation: caller-drawn keys)    -> tgo_select_by_keys
  *   3. Layers above L see only the kept tokens; no KV exists for dropped ones
  *                                                 -> tgo_compact_gather
  *   4. Token-gated attention: each kept token's score is added, scaled by a
@@ -161,6 +162,62 @@ int tgo_topk_select(const float* z, int32_t B, const int32_t* cu_seqlens, const 
         for (int32_t p = 0; p < s; ++p) kept[m++] = p;                     /* protected before the span */
         for (int32_t p = e; p < n; ++p) kept[m++] = p;                     /* protected after the span */
         qsort(kept, (size_t)m, sizeof(int32_t), cmp_int32);                /* keep original order */
+
+        for (int32_t i = 0; i < m; ++i) kept_idx[cu_kept[b] + i] = start + kept[i];
+        cu_kept[b + 1] = cu_kept[b] + m;
+        free(doc);
+        free(kept);
+    }
+    return 0;
+}
+
+/*
+ * Random-K selection (pages: the random-K selector ablation, a selector that
+ * keeps K document tokens at random instead of by gate score).  The random
+ * numbers are the caller's: one uint32 key per token; the K document tokens
+ * with the largest keys are kept (equal keys: lower index first), with the
+ * question protected and the kept rows in ascending order, exactly as in
+ * tgo_topk_select.  With i.i.d. uniform keys every K-subset of the document is
+ * equally likely.
+ */
+typedef struct {
+    int32_t idx;
+    uint32_t key;
+} keyed_token;
+
+static int cmp_key_rank(const void* pa, const void* pb) {
+    const keyed_token* a = (const keyed_token*)pa;
+    const keyed_token* b = (const keyed_token*)pb;
+    if (a->key != b->key) return a->key > b->key ? -1 : 1;
+    return (a->idx > b->idx) - (a->idx < b->idx);
+}
+
+int tgo_select_by_keys(const uint32_t* keys, int32_t B, const int32_t* cu_seqlens,
+                       const int32_t* doc_begin, const int32_t* doc_end, const int32_t* budget,
+                       int32_t* kept_idx, int32_t* cu_kept) {
+    if (!keys || !cu_seqlens || !doc_begin || !doc_end || !budget || !cu_kept || B < 0) return 1;
+    cu_kept[0] = 0;
+    for (int32_t b = 0; b < B; ++b) {
+        int32_t start = cu_seqlens[b];
+        int32_t n = cu_seqlens[b + 1] - start;
+        int32_t s = doc_begin[b], e = doc_end[b], K = budget[b];
+        if (n < 0 || s < 0 || e < s || e > n || K < 0) return 1;
+        int32_t n_doc = e - s;
+        int32_t k_keep = K < n_doc ? K : n_doc;
+
+        keyed_token* doc = (keyed_token*)malloc(sizeof(keyed_token) * (n_doc > 0 ? n_doc : 1));
+        int32_t* kept = (int32_t*)malloc(sizeof(int32_t) * (n > 0 ? n : 1));
+        for (int32_t i = 0; i < n_doc; ++i) {
+            doc[i].idx = s + i;
+            doc[i].key = keys[start + s + i];
+        }
+        qsort(doc, (size_t)n_doc, sizeof(keyed_token), cmp_key_rank);
+
+        int32_t m = 0;
+        for (int32_t i = 0; i < k_keep; ++i) kept[m++] = doc[i].idx;
+        for (int32_t p = 0; p < s; ++p) kept[m++] = p;
+        for (int32_t p = e; p < n; ++p) kept[m++] = p;
+        qsort(kept, (size_t)m, sizeof(int32_t), cmp_int32);
 
         for (int32_t i = 0; i < m; ++i) kept_idx[cu_kept[b] + i] = start + kept[i];
         cu_kept[b + 1] = cu_kept[b] + m;
