@@ -469,6 +469,18 @@ def run_extras(args):
     import ctypes
     st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     stage_us = {s: timed(lambda s=s: getattr(layer, s)(st), 20) for s in GatedLayer.STAGES}
+    # selection variants on the layer's scores: an 8-budget sweep in one launch vs
+    # eight single-budget launches, and random-K from caller-drawn keys
+    n_doc = np.asarray(inp.doc_end) - np.asarray(inp.doc_begin)
+    sweep = [[max(1, int(f * nd)) for nd in n_doc]
+             for f in (0.01, 0.02, 0.05, 0.0625, 0.1, 0.125, 0.25, 0.5)]
+    sweep_one = timed(lambda: tg.topk_select_multi(layer.z, inp.cu_seqlens, inp.doc_begin,
+                                                   inp.doc_end, sweep), 20)
+    sweep_sep = timed(lambda: [tg.topk_select(layer.z, inp.cu_seqlens, inp.doc_begin, inp.doc_end,
+                                              k) for k in sweep], 20)
+    keys = torch.from_numpy(gen.random_keys(w.total_tokens, seed=w.seed).view(np.int32)).to(dev)
+    rand_us = timed(lambda: tg.random_select(keys, inp.cu_seqlens, inp.doc_begin, inp.doc_end,
+                                             inp.budget), 20)
     ws = layer.workspace
     with_bias = timed(lambda: tg.gated_attention(layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host,
                                                  layer.logsig, layer.gain, layer.temp,
@@ -505,6 +517,9 @@ def run_extras(args):
         "ungated_attention": {"us": round(ungated, 2), "tflops": round(full_flops / ungated / 1e6, 1),
                               "frac_measured_bf16": round(full_flops / ungated / 1e6 / _peaks()["bf16"], 4)},
         "speedup_vs_ungated_attention": round(ungated / gated_total, 2),
+        "selection": {"budget_sweep_8_one_launch_us": round(sweep_one, 2),
+                      "budget_sweep_8_separate_launches_us": round(sweep_sep, 2),
+                      "random_k_us": round(rand_us, 2), "topk_us": round(stage_us["topk"], 2)},
         "memory_bytes": {
             "gated_step_allocated": int(gated_peak), "ungated_step_allocated": int(full_peak),
             "kv_gated": int(2 * sum(w.kept_lengths()) * w.n_kv_heads * dh * esz),

@@ -139,6 +139,42 @@ TG_API tg_status tg_topk_select(const float* z, int32_t batch, const int32_t* cu
                          const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
                          tg_stream_t stream);
 
+#define TG_MAX_BUDGETS 8
+
+/*
+ * Step 2 for a budget sweep: one scoring pass, several budgets (pages: the
+ * budget max_kept_prefill_tokens is a user choice; sweeping it reuses the
+ * gate's scores).  Budget q keeps, per prompt, exactly what tg_topk_select
+ * with budgets_h[q * batch .. q * batch + batch - 1] keeps; all budgets are
+ * selected in one launch from the same scores.
+ *   n_budgets     1 .. TG_MAX_BUDGETS
+ *   budgets_h     host [n_budgets][batch] document tokens to keep
+ *   kept_idx_out  host array of n_budgets device pointers, budget q's rows
+ *                 [M_q] (M_q = sum over prompts of its kept rows)
+ *   cu_kept_out   host array of n_budgets device pointers [batch+1] (entries
+ *                 may be NULL), or NULL
+ * Other arguments, order and limits as for tg_topk_select.
+ */
+TG_API tg_status tg_topk_select_multi(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                               const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                               int32_t n_budgets, const int32_t* budgets_h,
+                               int32_t* const* kept_idx_out, int32_t* const* cu_kept_out,
+                               tg_stream_t stream);
+
+/*
+ * Random-K selection (pages: the random-K selector ablation, which keeps K
+ * document tokens at random instead of by gate score).  The random numbers are
+ * the caller's: keys[total_tokens] uint32, one per token (for example i.i.d.
+ * uniform from a counter-based generator); the K document tokens with the
+ * largest keys are kept, equal keys by lower index, question protected, rows
+ * ascending -- the selection of tg_topk_select with the keys as scores.  With
+ * i.i.d. uniform keys every K-subset of the document is equally likely.
+ */
+TG_API tg_status tg_random_select(const uint32_t* keys, int32_t batch, const int32_t* cu_seqlens_h,
+                           const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                           const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
+                           tg_stream_t stream);
+
 /* One tensor to compact: rows of `row_elems` elements, pitch = row_elems. */
 typedef struct {
     const void* src;     /* device [total_tokens, row_elems] */

@@ -24,7 +24,7 @@ __all__ = [
     "TG_BF16", "TG_FP32", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "TokenGateError",
     "library", "kept_offsets", "gate_score", "topk_select", "compact_gather", "gated_attention",
     "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
-    "attention_kernel",
+    "attention_kernel", "topk_select_multi", "random_select",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -39,8 +39,9 @@ EXPORTED_SYMBOLS = (
     "tg_status_string", "tg_last_error_message", "tg_version", "tg_device_status",
     "tg_kept_offsets", "tg_gate_score", "tg_topk_select", "tg_compact_gather",
     "tg_gated_attention", "tg_attention_workspace_bytes", "tg_attention_kernel",
-    "tg_gated_attention_noalloc",
+    "tg_gated_attention_noalloc", "tg_topk_select_multi", "tg_random_select",
 )
+MAX_BUDGETS = 8
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
                 3: "attn_pair_kernel"}
 
@@ -81,6 +82,9 @@ def library():
     L.tg_gate_score.argtypes = [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, _i32, _vp, _f32, _vp,
                                 _i32, _vp]
     L.tg_topk_select.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp]
+    L.tg_topk_select_multi.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32, _i32p,
+                                       ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp]
+    L.tg_random_select.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp]
     L.tg_compact_gather.argtypes = [_vp, _i64, _i32, _i32p, _i32p, _i32p, _i32p, ctypes.c_int,
                                     ctypes.POINTER(GatherTensor), _i32, _i32, ctypes.c_double,
                                     _vp, _vp, _vp]
@@ -188,6 +192,50 @@ def topk_select(z, cu_seqlens, doc_begin, doc_end, budget, kept_idx=None, cu_kep
         cu_kept = torch.empty(len(s) + 1, dtype=torch.int32, device=z.device)
     _check("tg_topk_select", library().tg_topk_select(
         _ptr(z), len(s), cu_p, s_p, e_p, k_p, _ptr(kept_idx), _ptr(cu_kept), _stream(z.device)))
+    return kept_idx, cu_kept, host
+
+
+def topk_select_multi(z, cu_seqlens, doc_begin, doc_end, budgets):
+    """Top-K for a budget sweep from one score vector: budgets is a list of
+    per-prompt budget lists (at most MAX_BUDGETS).  One launch.
+
+    Returns a list of (kept_idx [M_q] device, cu_kept [B+1] device, cu_kept_host).
+    """
+    _need_cuda(z)
+    cu, cu_p = _host_i32(cu_seqlens)
+    s, s_p = _host_i32(doc_begin)
+    e, e_p = _host_i32(doc_end)
+    ks = np.ascontiguousarray(np.asarray(budgets, dtype=np.int32).reshape(len(budgets), len(s)))
+    outs, kept_ptrs, cu_ptrs = [], (_vp * len(ks))(), (_vp * len(ks))()
+    for q, k in enumerate(ks):
+        host = kept_offsets(cu, s, e, k)
+        M = int(host[-1])
+        kept = torch.empty(max(M, 1), dtype=torch.int32, device=z.device)[:M]
+        cuk = torch.empty(len(s) + 1, dtype=torch.int32, device=z.device)
+        kept_ptrs[q], cu_ptrs[q] = kept.data_ptr() if M else None, cuk.data_ptr()
+        outs.append((kept, cuk, host))
+    _check("tg_topk_select_multi", library().tg_topk_select_multi(
+        _ptr(z), len(s), cu_p, s_p, e_p, len(ks), ks.ctypes.data_as(_i32p), kept_ptrs, cu_ptrs,
+        _stream(z.device)))
+    return outs
+
+
+def random_select(keys, cu_seqlens, doc_begin, doc_end, budget):
+    """Random-K selection from caller-drawn uint32 keys (a device tensor of
+    torch.int32 holding the key bits, one per token): the K document tokens with
+    the largest keys, question kept.  Returns (kept_idx, cu_kept, cu_kept_host)."""
+    _need_cuda(keys)
+    cu, cu_p = _host_i32(cu_seqlens)
+    s, s_p = _host_i32(doc_begin)
+    e, e_p = _host_i32(doc_end)
+    k, k_p = _host_i32(budget)
+    host = kept_offsets(cu, s, e, k)
+    M = int(host[-1])
+    kept_idx = torch.empty(max(M, 1), dtype=torch.int32, device=keys.device)[:M]
+    cu_kept = torch.empty(len(s) + 1, dtype=torch.int32, device=keys.device)
+    _check("tg_random_select", library().tg_random_select(
+        _ptr(keys), len(s), cu_p, s_p, e_p, k_p, _ptr(kept_idx), _ptr(cu_kept),
+        _stream(keys.device)))
     return kept_idx, cu_kept, host
 
 

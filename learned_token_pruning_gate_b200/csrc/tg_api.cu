@@ -246,7 +246,52 @@ tg_status tg_topk_select(const float* z, int32_t batch, const int32_t* cu_seqlen
   if (t.start[batch] > 0 && !z) return set_error(TG_ERR_INVALID_ARG, "z is null");
   if (max_len > 360448)
     return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens exceeds 360448", max_len);
-  return launch_topk(z, t, max_len, kept_idx_out, cu_kept_out,
+  return launch_topk(z, nullptr, &t, 1, max_len, &kept_idx_out, &cu_kept_out,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+tg_status tg_topk_select_multi(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                               const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                               int32_t n_budgets, const int32_t* budgets_h,
+                               int32_t* const* kept_idx_out, int32_t* const* cu_kept_out,
+                               tg_stream_t stream) {
+  if (n_budgets < 1 || n_budgets > TG_MAX_BUDGETS)
+    return set_error(TG_ERR_INVALID_ARG, "n_budgets=%d (1..%d)", n_budgets, TG_MAX_BUDGETS);
+  if (!budgets_h || !kept_idx_out) return set_error(TG_ERR_INVALID_ARG, "null budget array");
+  static thread_local PromptTable t[TG_MAX_BUDGETS];
+  int max_len = 0;
+  for (int q = 0; q < n_budgets; ++q) {
+    tg_status r = build_table(batch, cu_seqlens_h, doc_begin_h, doc_end_h,
+                              budgets_h + static_cast<int64_t>(q) * (batch > 0 ? batch : 0), &t[q],
+                              &max_len, nullptr);
+    if (r != TG_OK) return r;
+    if (batch > 0 && t[q].kept_start[batch] > 0 && !kept_idx_out[q])
+      return set_error(TG_ERR_INVALID_ARG, "kept_idx_out[%d] is null", q);
+  }
+  if (batch == 0) return TG_OK;
+  if (t[0].start[batch] > 0 && !z) return set_error(TG_ERR_INVALID_ARG, "z is null");
+  if (max_len > 360448)
+    return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens exceeds 360448", max_len);
+  return launch_topk(z, nullptr, t, n_budgets, max_len, kept_idx_out, cu_kept_out,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+tg_status tg_random_select(const uint32_t* keys, int32_t batch, const int32_t* cu_seqlens_h,
+                           const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                           const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
+                           tg_stream_t stream) {
+  PromptTable t;
+  int max_len = 0;
+  tg_status r = build_table(batch, cu_seqlens_h, doc_begin_h, doc_end_h, budget_h, &t, &max_len,
+                            nullptr);
+  if (r != TG_OK) return r;
+  if (batch == 0) return TG_OK;
+  if (t.kept_start[batch] > 0 && !kept_idx_out)
+    return set_error(TG_ERR_INVALID_ARG, "kept_idx_out is null");
+  if (t.start[batch] > 0 && !keys) return set_error(TG_ERR_INVALID_ARG, "keys is null");
+  if (max_len > 360448)
+    return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens exceeds 360448", max_len);
+  return launch_topk(nullptr, keys, &t, 1, max_len, &kept_idx_out, &cu_kept_out,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -46,8 +46,9 @@ tg_status launch_gate_simt(const void* h, tg_dtype dt, int64_t n, int d, const v
                            cudaStream_t st);
 tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const float* b1, int dg,
                          const float* w2, float b2, float* z, cudaStream_t st);
-tg_status launch_topk(const float* z, const PromptTable& pt, int max_len, int32_t* kept_idx,
-                      int32_t* cu_kept, cudaStream_t st);
+tg_status launch_topk(const float* z, const uint32_t* keys, const PromptTable* tables,
+                      int n_budgets, int max_len, int32_t* const* kept_idx,
+                      int32_t* const* cu_kept, cudaStream_t st);
 tg_status launch_gather(const int32_t* kept_idx, int64_t m_total, const PromptTable& pt,
                         tg_dtype dt, const tg_gather_tensor* tensors, int n_tensors, int head_dim,
                         double theta, const float* z, float* logsig, cudaStream_t st);

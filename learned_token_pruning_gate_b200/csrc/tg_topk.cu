@@ -2,8 +2,11 @@
 // (TokenGate: "a top-K selector keeps the highest-scoring tokens"; "only the
 // document part of the prompt is pruned, the question is never touched").
 //
-// One cluster of 8 CTAs per prompt, one launch; each CTA owns a contiguous
-// eighth of the prompt.
+// One cluster of 8 CTAs per (budget, prompt), one launch; each CTA owns a
+// contiguous eighth of the prompt.  Several budgets (a budget sweep served by
+// one scoring pass) select from the same scores in the same launch.  The keys
+// are either fp32 gate scores or caller-drawn uint32 keys (the random-K
+// selector ablation): larger first, lower index on ties, in both cases.
 //  1. Each CTA caches its slice of the scores in shared memory as
 //     order-preserving 32-bit keys (padded by one word per 32 so both strided
 //     and per-thread-contiguous walks are free of bank conflicts) and builds the
@@ -34,12 +37,15 @@ constexpr int kBins = 2048;
 constexpr int kMaxCluster = 8;
 
 struct TopkParams {
-  PromptTable pt;
-  const float* z;
-  int32_t* kept_idx;
-  int32_t* cu_kept;
+  PromptTable pt;  // prompt offsets and document spans (budget-independent fields)
+  int32_t k_keep[TG_MAX_BUDGETS][kMaxBatch];          // per budget: min(K, n_doc)
+  int32_t kept_start[TG_MAX_BUDGETS][kMaxBatch + 1];  // per budget: cu_kept
+  int32_t* kept_idx[TG_MAX_BUDGETS];
+  int32_t* cu_kept[TG_MAX_BUDGETS];
+  const float* z;      // scores (kKeys = false)
+  const uint32_t* keys;  // caller keys (kKeys = true)
   uint32_t* status;
-  int32_t cluster;  // CTAs per prompt
+  int32_t cluster;  // CTAs per (budget, prompt)
 };
 
 // Order-preserving key: larger score -> larger key; -0.0 maps to +0.0; NaN maps
@@ -84,6 +90,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
   return r;
 }
 
+template <bool kKeys>
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant__ TopkParams p) {
   extern __shared__ uint32_t s_keys[];  // padded layout
   __shared__ uint32_t s_hist[kBins];           // this CTA's histogram of the current pass
@@ -95,13 +102,14 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = p.cluster;
   const int r = static_cast<int>(cluster.block_rank());
-  const int b = blockIdx.x / CL;
+  const int q = (blockIdx.x / CL) / p.pt.batch;  // budget
+  const int b = (blockIdx.x / CL) - q * p.pt.batch;
   const int tid = threadIdx.x;
 
   const int32_t start = p.pt.start[b];
   const int32_t n = p.pt.start[b + 1] - start;
   const int32_t ds = p.pt.doc_begin[b], de = p.pt.doc_end[b];
-  const int32_t kk = p.pt.k_keep[b];
+  const int32_t kk = p.k_keep[q][b];
   const int32_t n_doc = de - ds;
   const int32_t chunk = (n + CL - 1) / CL;
   const int32_t lo = min(n, r * chunk);
@@ -117,7 +125,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
   __syncthreads();
   // keys into shared memory; pass-0 histogram (top 11 bits) on the way
   for (int i = tid; i < len; i += kThreads) {
-    const uint32_t key = order_key(__ldg(p.z + start + lo + i));
+    const uint32_t key =
+        kKeys ? __ldg(p.keys + start + lo + i) : order_key(__ldg(p.z + start + lo + i));
     s_keys[padded(i)] = key;
     const int32_t pos = lo + i;
     if (mode == 2 && pos >= ds && pos < de) atomicAdd(&s_hist[key >> 21], 1u);
@@ -220,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
   const uint32_t need_here = need > peq ? need - peq : 0u;  // ties still to take in this CTA
   uint32_t out_pos = pgt + min(peq, need) + gt_before + min(need_here, eq_before);
   uint32_t tie_rank = eq_before;  // ties before this thread inside the CTA
-  int32_t* out = p.kept_idx + p.pt.kept_start[b];
-  const uint32_t m_b = static_cast<uint32_t>(p.pt.kept_start[b + 1] - p.pt.kept_start[b]);
+  int32_t* out = p.kept_idx[q] + p.kept_start[q][b];
+  const uint32_t m_b = static_cast<uint32_t>(p.kept_start[q][b + 1] - p.kept_start[q][b]);
   for (int32_t i = tlo; i < thi; ++i) {
     const int32_t pos = lo + i;
     const bool doc = pos >= ds && pos < de;
@@ -237,21 +246,28 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
       ++out_pos;
     }
   }
-  if (p.cu_kept && r == 0 && tid == 0) {
-    p.cu_kept[b + 1] = p.pt.kept_start[b + 1];
-    if (b == 0) p.cu_kept[0] = 0;
+  if (p.cu_kept[q] && r == 0 && tid == 0) {
+    p.cu_kept[q][b + 1] = p.kept_start[q][b + 1];
+    if (b == 0) p.cu_kept[q][0] = 0;
   }
 }
 
 }  // namespace
 
-tg_status launch_topk(const float* z, const PromptTable& pt, int max_len, int32_t* kept_idx,
-                      int32_t* cu_kept, cudaStream_t st) {
-  TopkParams p;
-  p.pt = pt;
+tg_status launch_topk(const float* z, const uint32_t* keys, const PromptTable* tables,
+                      int n_budgets, int max_len, int32_t* const* kept_idx,
+                      int32_t* const* cu_kept, cudaStream_t st) {
+  static thread_local TopkParams p;  // ~11 KB: kept off the stack
+  memset(&p, 0, sizeof(p));
+  p.pt = tables[0];
+  for (int q = 0; q < n_budgets; ++q) {
+    for (int b = 0; b < tables[q].batch; ++b) p.k_keep[q][b] = tables[q].k_keep[b];
+    for (int b = 0; b <= tables[q].batch; ++b) p.kept_start[q][b] = tables[q].kept_start[b];
+    p.kept_idx[q] = kept_idx[q];
+    p.cu_kept[q] = cu_kept ? cu_kept[q] : nullptr;
+  }
   p.z = z;
-  p.kept_idx = kept_idx;
-  p.cu_kept = cu_kept;
+  p.keys = keys;
   p.status = device_status_word();
   if (!p.status) return set_error(TG_ERR_CUDA, "device status word unavailable");
   const int cl = kMaxCluster;  // latency-bound: spread every prompt over 8 SMs
@@ -260,13 +276,14 @@ tg_status launch_topk(const float* z, const PromptTable& pt, int max_len, int32_
     return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens is too long for top-K", max_len);
   p.cluster = cl;
   const size_t dyn = static_cast<size_t>(padded(slice > 0 ? slice : 1) + 1) * sizeof(uint32_t);
+  auto kernel = keys ? topk_kernel<true> : topk_kernel<false>;
   tg_status r = cuda_check(
-      cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(dyn)),
       "topk smem attribute");
   if (r != TG_OK) return r;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(pt.batch * cl));
+  cfg.gridDim = dim3(static_cast<unsigned>(n_budgets * tables[0].batch * cl));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = dyn;
   cfg.stream = st;
@@ -277,7 +294,7 @@ tg_status launch_topk(const float* z, const PromptTable& pt, int max_len, int32_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, topk_kernel, p), "topk launch");
+  return cuda_check(cudaLaunchKernelEx(&cfg, kernel, p), "topk launch");
 }
 
 }  // namespace tg

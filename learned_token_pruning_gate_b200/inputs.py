@@ -163,6 +163,15 @@ def make_inputs(w: Workload, with_qkv: bool = True) -> Inputs:
                   gain, temp)
 
 
+def random_keys(n: int, seed: int, bits: int = 32) -> np.ndarray:
+    """i.i.d. uniform uint32 keys from a counter-based generator (Philox): the
+    random numbers the random-K selector draws.  bits < 32 leaves only the low
+    bits random, to plant many exact ties."""
+    rng = np.random.Generator(np.random.Philox(seed))
+    k = rng.integers(0, 1 << 32, n, dtype=np.uint64).astype(np.uint32)
+    return k & np.uint32((1 << bits) - 1) if bits < 32 else k
+
+
 def random_scores(n: int, seed: int, ties: bool = True, specials: bool = True) -> np.ndarray:
     """fp32 gate-score-like values with planted exact ties, +-0.0, +-inf and NaN."""
     rng = np.random.Generator(np.random.Philox(seed))

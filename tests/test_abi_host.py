@@ -218,3 +218,27 @@ def test_no_gpu_means_cuda_error_not_crash(L):
         pytest.skip("a GPU is present")
     bits = ctypes.c_uint32(0)
     assert L.tg_device_status(None, ctypes.byref(bits)) == CUDA
+
+
+def test_budget_sweep_and_random_select_validation(L):
+    cu, cu_p = _arr([0, 10])
+    s, s_p = _arr([2])
+    e, e_p = _arr([8])
+    ks, ks_p = _arr([3, 4])
+    ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    f = L.tg_topk_select_multi
+    assert f(FAKE, 1, cu_p, s_p, e_p, 0, ks_p, ptrs, None, None) == INVALID   # no budget
+    assert f(FAKE, 1, cu_p, s_p, e_p, 9, ks_p, ptrs, None, None) == INVALID   # > TG_MAX_BUDGETS
+    assert f(FAKE, 1, cu_p, s_p, e_p, 2, None, ptrs, None, None) == INVALID
+    nulls = (ctypes.c_void_p * 2)(FAKE, None)
+    assert f(FAKE, 1, cu_p, s_p, e_p, 2, ks_p, nulls, None, None) == INVALID  # budget 1 output
+    bad, bad_p = _arr([3, -1])
+    assert f(FAKE, 1, cu_p, s_p, e_p, 2, bad_p, ptrs, None, None) == INVALID  # negative budget
+    assert f(None, 1, cu_p, s_p, e_p, 2, ks_p, ptrs, None, None) == INVALID   # scores
+    r = L.tg_random_select
+    k1, k1_p = _arr([3])
+    assert r(None, 1, cu_p, s_p, e_p, k1_p, FAKE, FAKE, None) == INVALID      # keys
+    assert r(FAKE, 1, cu_p, s_p, e_p, k1_p, None, FAKE, None) == INVALID      # output
+    big, big_p = _arr([0, 400000])
+    s0, s0_p = _arr([0])
+    assert r(FAKE, 1, big_p, s0_p, s0_p, k1_p, FAKE, FAKE, None) == UNSUP     # too long

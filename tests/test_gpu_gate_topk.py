@@ -129,3 +129,49 @@ def test_topk_full_size(oracle, name, seed):
     e = np.array([n - q for n, q in zip(w.seqlens, w.question)], np.int32)
     z = gen.random_scores(int(cu[-1]), seed=seed, specials=False)
     _topk_both(oracle, z, cu, np.zeros(w.batch, np.int32), e, np.array(w.budgets, np.int32))
+
+
+# ---- random-K selection (caller-drawn keys) and budget sweeps ---------------------
+
+def _varlen(seed, lens):
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    s, e = [], []
+    for n in lens:
+        a = int(rng.integers(0, max(n // 4, 1))) if n else 0
+        b = int(rng.integers(max(a, n - n // 4), n + 1)) if n else 0
+        s.append(a)
+        e.append(b)
+    return cu, np.array(s, np.int32), np.array(e, np.int32)
+
+
+@pytest.mark.parametrize("lens,bits", [([1], 32), ([1000], 32), ([4097], 3), ([16384], 32),
+                                       ([131072], 32), ([5, 0, 300, 1, 2049], 32),
+                                       ([700, 900], 1)])
+def test_random_select_bit_exact(oracle, lens, bits):
+    cu, s, e = _varlen(len(lens) + bits, lens)
+    keys = gen.random_keys(int(cu[-1]), seed=sum(lens) + bits, bits=bits)
+    rng = np.random.default_rng(bits)
+    for kfrac in (0.0, 0.1, 0.5, 1.0, 2.0):
+        k = np.array([int(kfrac * (b - a)) for a, b in zip(s, e)], np.int32)
+        kk, ck, _ = tg.random_select(torch.from_numpy(keys.view(np.int32)).cuda(), cu, s, e, k)
+        ref, ref_cu = oracle.select_by_keys(keys, cu, s, e, k)
+        assert ck.cpu().numpy().tolist() == ref_cu.tolist()
+        np.testing.assert_array_equal(kk.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("lens", [[16384], [5, 0, 300, 1, 2049, 8192], [131072]])
+def test_topk_budget_sweep_bit_exact(oracle, lens):
+    """One launch, up to eight budgets from the same scores: each budget's
+    kept rows equal the oracle's top-K with that budget."""
+    cu, s, e = _varlen(7, lens)
+    z = gen.random_scores(int(cu[-1]), seed=len(lens))
+    n_doc = e - s
+    fracs = [0.0, 0.01, 0.125, 0.3, 0.5, 0.9, 1.0, 1.5]
+    budgets = [[int(f * nd) for nd in n_doc] for f in fracs]
+    outs = tg.topk_select_multi(torch.from_numpy(z).cuda(), cu, s, e, budgets)
+    assert len(outs) == len(budgets)
+    for (kk, ck, host), k in zip(outs, budgets):
+        ref, ref_cu = oracle.topk_select(z, cu, s, e, k)
+        assert ck.cpu().numpy().tolist() == ref_cu.tolist() == host.tolist()
+        np.testing.assert_array_equal(kk.cpu().numpy(), ref)
