@@ -583,21 +583,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                                __uint_as_float(orow[4 * v4 + 2]) * inv,
                                __uint_as_float(orow[4 * v4 + 3]) * inv));
         }
-        __stcg(p.part_lse + ((w.slot + w.c) * 2 + x) * 128 + rl, m + log2f(l));
-        tc_fence_before();
-        mbar_arrive(bar(kOFree + x));
-        // publish, then count arrivals; the last chunk to arrive merges
+        const float lse_own = m + log2f(l);
+        __stcg(p.part_lse + ((w.slot + w.c) * 2 + x) * 128 + rl, lse_own);
+        // publish, then count arrivals; the last chunk to arrive merges.  O stays
+        // in TMEM until then: the merge reads this chunk's own part from there.
         __threadfence();
         named_barrier(1 + x, 128);
         if (rl == 0) last_flag[x] = atomicAdd(p.part_cnt + w.slot * 2 + x, 1) == w.n - 1;
         named_barrier(1 + x, 128);
         if (last_flag[x]) {
           __threadfence();
+          // weights in chunk order (the own LSE is the value stored above)
           float lc[kMaxChunks], wc[kMaxChunks];
           float mx = -INFINITY;
 #pragma unroll
           for (int cc = 0; cc < kMaxChunks; ++cc) {
-            lc[cc] = cc < w.n ? __ldcg(p.part_lse + ((w.slot + cc) * 2 + x) * 128 + rl) : -INFINITY;
+            lc[cc] = cc >= w.n ? -INFINITY
+                     : cc == w.c ? lse_own
+                                 : __ldcg(p.part_lse + ((w.slot + cc) * 2 + x) * 128 + rl);
             mx = fmaxf(mx, lc[cc]);
           }
           float wsum = 0.0f;
@@ -611,38 +614,68 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < kMaxChunks; ++cc) wc[cc] *= winv;
           const float4* pb = p.part_o + static_cast<int64_t>(w.slot * 2 + x) * kV4 * 128 + rl;
           const int64_t slot_stride = 2 * kV4 * 128;
+          // The sum runs over the chunks in index order with the very values
+          // each chunk stored, so it does not depend on which chunk is last.
+          // Two 32-column blocks per round: every partial read of a round is in
+          // flight at once.
 #pragma unroll 1
-          for (int c = 0; c < DH / 32; ++c) {
-            float acc[32];
+          for (int c2 = 0; c2 < DH / 32; c2 += 2) {
+            float acc[2][32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[h][e] = 0.0f;
 #pragma unroll 1
             for (int cc = 0; cc < w.n; ++cc) {
+              if (cc == w.c) {
 #pragma unroll
-              for (int v4 = 0; v4 < 8; ++v4) {
-                const float4 a = __ldcg(pb + cc * slot_stride + (c * 8 + v4) * 128);
-                acc[4 * v4] = fmaf(wc[cc], a.x, acc[4 * v4]);
-                acc[4 * v4 + 1] = fmaf(wc[cc], a.y, acc[4 * v4 + 1]);
-                acc[4 * v4 + 2] = fmaf(wc[cc], a.z, acc[4 * v4 + 2]);
-                acc[4 * v4 + 3] = fmaf(wc[cc], a.w, acc[4 * v4 + 3]);
+                for (int h = 0; h < 2; ++h) {
+                  uint32_t orow[32];
+                  tmem_ld32(t_o + (c2 + h) * 32, orow);
+                  tmem_ld_wait(orow);
+#pragma unroll
+                  for (int e = 0; e < 32; ++e)
+                    acc[h][e] = fmaf(wc[cc], __uint_as_float(orow[e]) * inv, acc[h][e]);
+                }
+              } else {
+                float4 a[2][8];
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                  for (int v4 = 0; v4 < 8; ++v4)
+                    a[h][v4] = __ldcg(pb + cc * slot_stride + ((c2 + h) * 8 + v4) * 128);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                  for (int v4 = 0; v4 < 8; ++v4) {
+                    acc[h][4 * v4] = fmaf(wc[cc], a[h][v4].x, acc[h][4 * v4]);
+                    acc[h][4 * v4 + 1] = fmaf(wc[cc], a[h][v4].y, acc[h][4 * v4 + 1]);
+                    acc[h][4 * v4 + 2] = fmaf(wc[cc], a[h][v4].z, acc[h][4 * v4 + 2]);
+                    acc[h][4 * v4 + 3] = fmaf(wc[cc], a[h][v4].w, acc[h][4 * v4 + 3]);
+                  }
               }
             }
             if (qi < len) {
-              uint32_t pkd[16];
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                __nv_bfloat162 pp = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
-                pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
+              for (int h = 0; h < 2; ++h) {
+                uint32_t pkd[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  __nv_bfloat162 pp = __floats2bfloat162_rn(acc[h][2 * e], acc[h][2 * e + 1]);
+                  pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(out + (c2 + h) * 32);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                  dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
               }
-              uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-              for (int v4 = 0; v4 < 4; ++v4)
-                dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
             }
           }
           if (p.lse && qi < len)
             p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (mx + log2f(wsum)) * kLn2;
         }
+        tc_fence_before();
+        mbar_arrive(bar(kOFree + x));  // O may now be overwritten by the next unit
       }
     }
   }
