@@ -490,25 +490,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           alpha = exp2_approx(m - mx);
           m = mx;
         }
-        // The previous tile's P.V is complete (this tile's S commit tracked it), so
-        // O may be rescaled in place.  Warp-uniform: tcgen05.ld/st are collective.
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
-            uint32_t orow[32];
-            tmem_ld32(t_o + c * 32, orow);
-            tmem_ld_wait(orow);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float2 v2 = __fmul2_rn(
-                  make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
-                  make_float2(alpha, alpha));
-              orow[e] = __float_as_uint(v2.x);
-              orow[e + 1] = __float_as_uint(v2.y);
-            }
-            tmem_st32(t_o + c * 32, orow);
-          }
-        }
         // p = 2^(t - m), row sum, and P (bf16 pairs) over the first 64 columns of S,
         // 32 keys (16 columns) at a time
         const float2 nm2 = make_float2(-m, -m);
@@ -528,6 +509,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(t_s + c * 16, pk);
         }
         l = fmaf(l, alpha, (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
+        // The previous tile's P.V is complete (this tile's S commit tracked it) and
+        // this tile's is not issued before P is marked full, so O may be rescaled
+        // in place: done after the exponentials, when S holds no registers.
+        // Warp-uniform: tcgen05.ld/st are collective.
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t orow[32];
+            tmem_ld32(t_o + c * 32, orow);
+            tmem_ld_wait(orow);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v2 = __fmul2_rn(
+                  make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
+                  make_float2(alpha, alpha));
+              orow[e] = __float_as_uint(v2.x);
+              orow[e + 1] = __float_as_uint(v2.y);
+            }
+            tmem_st32(t_o + c * 32, orow);
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(kPFull + x));
