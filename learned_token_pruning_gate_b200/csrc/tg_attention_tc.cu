@@ -101,8 +101,12 @@ struct Lay {
   static constexpr uint32_t kQb = kTile;
   static constexpr uint32_t kK = 2 * kTile;
   static constexpr uint32_t kV = kK + kStages * kTile;
-  static constexpr uint32_t kBias = kV + kStages * kTile;  // [2 heads][2 parity][128] fp32
-  static constexpr uint32_t kBars = kBias + 2 * 2 * 128 * 4;
+  // operands of the bias step of S: A_a, A_b (per head) and B_0, B_1 (per key
+  // tile, by tile parity), each 128 rows x 16 bf16, K-major without swizzle:
+  // rows of 16 bytes for k = 0..7, then 2 KB of zeros for k = 8..15
+  static constexpr uint32_t kAugTile = 4096;
+  static constexpr uint32_t kAug = kV + kStages * kTile;
+  static constexpr uint32_t kBars = kAug + 4 * kAugTile;
   static constexpr uint32_t kMisc = kBars + 32 * 8;
   static constexpr uint32_t kTotal = kMisc + 16;  // tmem slot, abort flag, last-chunk flags[2]
   static constexpr uint32_t kDynSmem = kTotal + 1024;
@@ -117,6 +121,7 @@ enum {
   kOFull = 6,   // [2]
   kOFree = 8,   // [2]
   kKFull = 10,  // [stages]
+  kAugFull = 22,  // [2] bias operands of an item's first tile written
   kDrain = 31,  // MMA completion on the way out after an abort
 };
 
@@ -212,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
-  float* s_bias = reinterpret_cast<float*>(smem + L::kBias);
+  static_assert(kKFull + 3 * S <= kAugFull, "barrier slots");
+  uint8_t* s_aug = smem + L::kAug;
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) { return smem_u32(bars + i); };
   auto k_full = [&](int s) { return bar(kKFull + s); };
@@ -228,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kPFull + x), 128);
       mbar_init(bar(kOFull + x), 1);
       mbar_init(bar(kOFree + x), 128);
+      mbar_init(bar(kAugFull + x), 128);
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(k_full(s), 1);
@@ -245,6 +252,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
+  // the zero halves (k = 8..15) of the bias operands are never written again
+  for (int i = threadIdx.x; i < static_cast<int>(4 * L::kAugTile / 16); i += kThreads)
+    reinterpret_cast<uint4*>(s_aug)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -312,7 +323,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t d_q[2] = {sw128_desc(sb + L::kQa, 16, 1024), sw128_desc(sb + L::kQb, 16, 1024)};
       const uint64_t d_k0 = sw128_desc(sb + L::kK, 16, 1024);
       const uint64_t d_v0 = sw128_desc(sb + L::kV, L::kBox, 1024);
-      auto issue_s = [&](int x, int s) {
+      const uint64_t d_aug_a = nosw_desc(sb + L::kAug, 2048, 128);
+      const uint64_t d_aug_b = nosw_desc(sb + L::kAug + 2 * L::kAugTile, 2048, 128);
+      constexpr uint32_t kAug16 = L::kAugTile >> 4;
+      // S_x = Q_x K^T + A_x B^T for head x, K tile in stage s, bias operand B of
+      // tile parity tp
+      auto issue_s = [&](int x, int s, uint32_t tp) {
         const uint64_t dq = d_q[x];
         const uint64_t dk = d_k0 + ((s * L::kTile) >> 4);
         const uint32_t ts = tmem + x * 128;
@@ -322,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t off = (kk >> 2) * kBox16 + (kk & 3) * 2;
           umma_ss(ts, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
+        umma_ss(ts, d_aug_a + x * kAug16, d_aug_b + tp * kAug16, idesc_qk, 1u);
         umma_commit(bar(kSFull + x));
       };
       // O_x (+)= P_x V with the V tile in stage s
@@ -334,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       int rs = 0;
       uint32_t rph = 0, q_waits = 0, p_waits[2] = {0, 0}, of_waits[2] = {0, 0};
+      uint32_t aug_waits[2] = {0, 0}, tile_base = 0;  // tiles of earlier units
       bool ok = true;
       for (int round = 0; ok; ++round) {
         const int u = snake_unit(round, blockIdx.x, gridDim.x);
@@ -343,9 +361,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_kv = w.j1 - w.j0;
         if (!(ok = wt(bar(kQFull), q_waits++ & 1))) break;
         if (!(ok = wt(k_full(rs), rph))) break;
+        if (!(ok = wt(bar(kAugFull + 0), aug_waits[0]++ & 1))) break;
         tc_fence_after();
-        issue_s(0, rs);
-        if (it.has_b) issue_s(1, rs);
+        issue_s(0, rs, tile_base & 1);
+        if (it.has_b) {
+          if (!(ok = wt(bar(kAugFull + 1), aug_waits[1]++ & 1))) break;
+          tc_fence_after();
+          issue_s(1, rs, tile_base & 1);
+        }
         if (n_kv == 1) umma_commit(bar(kQEmpty));
         for (int j = 0; ok && j < n_kv; ++j) {
           int ns = rs + 1;
@@ -365,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (more) {
             if (!(ok = wt(k_full(ns), nph))) break;
             tc_fence_after();
-            issue_s(0, ns);
+            issue_s(0, ns, (tile_base + j + 1) & 1);
             if (!it.has_b && j + 2 == n_kv) umma_commit(bar(kQEmpty));
           }
           // head b: P_b(j) V_j, then S_b(j+1)
@@ -378,12 +401,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           umma_commit(kv_empty(rs));  // V_j (and K_j) no longer needed once these finish
           if (more && it.has_b) {
-            issue_s(1, ns);
+            issue_s(1, ns, (tile_base + j + 1) & 1);
             if (j + 2 == n_kv) umma_commit(bar(kQEmpty));
           }
           rs = ns;
           rph = nph;
         }
+        tile_base += n_kv;
       }
     }
     __syncwarp();
@@ -409,23 +433,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t len = p.kept_start[it.b + 1] - kstart;
       const int n_kv = w.j1 - w.j0;
       const float scale = kLog2e / (sqrtf(static_cast<float>(DH)) * __ldg(p.temp + head));
-      const float gl = __ldg(p.gain + head) * kLog2e;
       const float2 sc2 = make_float2(scale, scale);
+      // Bias operands.  S = Q K^T + A B^T with A row = [c_hi, c_lo, c_hi, c_lo] and
+      // B row j = [l_hi, l_hi, l_lo, l_lo] (bf16 halves of c = g_h log2e / scale and
+      // of the key's log-gate l_j), so S_ij = q.k + c l_j to about 2^-16 relative
+      // and scale * S is the log2-domain logit.  Key rows beyond the prompt and
+      // question keys carry l = 0.
+      {
+        const float cb = p.logsig ? __ldg(p.gain + head) * kLog2e / scale : 0.0f;
+        const __nv_bfloat16 c_hi = __float2bfloat16_rn(cb);
+        const __nv_bfloat16 c_lo = __float2bfloat16_rn(cb - __bfloat162float(c_hi));
+        const __nv_bfloat162 ca = __halves2bfloat162(c_hi, c_lo);
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(&ca);
+        *reinterpret_cast<uint4*>(s_aug + x * L::kAugTile + rl * 16) = make_uint4(cw, cw, 0u, 0u);
+      }
+      auto load_l = [&](int key) {  // the key's log-gate (key index in the prompt)
+        return (p.logsig && key < len) ? __ldg(p.logsig + kstart + key) : 0.0f;
+      };
+      auto aug_row = [](float lj) {  // bias operand row of a key
+        lj = fmaxf(lj, -1e30f);
+        const __nv_bfloat16 l_hi = __float2bfloat16_rn(lj);
+        const __nv_bfloat16 l_lo = __float2bfloat16_rn(lj - __bfloat162float(l_hi));
+        const __nv_bfloat162 h2 = __halves2bfloat162(l_hi, l_hi), o2 = __halves2bfloat162(l_lo, l_lo);
+        return make_uint4(*reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&o2),
+                          0u, 0u);
+      };
+      auto aug_b_row = [&](uint32_t tile) {
+        return reinterpret_cast<uint4*>(s_aug + (2 + (tile & 1)) * L::kAugTile + rl * 16);
+      };
+      // head a's warpgroup writes B for every tile: the first one now, tile j + 1
+      // while tile j is in softmax (after S_j is complete, so both heads' S of the
+      // tile that used the same parity are done); the log-gates are loaded one
+      // tile ahead of their use
+      float next_l = 0.0f;
+      if (x == 0) {
+        *aug_b_row(tile_ctr) = aug_row(load_l(w.j0 * kBN + rl));
+        if (n_kv > 1) next_l = load_l((w.j0 + 1) * kBN + rl);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kAugFull + x));
       float m = -INFINITY, l = 0.0f;
-      // this thread's key of the next tile's bias, loaded one tile ahead
-      const int key0 = w.j0 * kBN + rl;
-      float next_bias = (p.logsig && key0 < len) ? gl * __ldg(p.logsig + kstart + key0) : 0.0f;
       for (int j = 0; j < n_kv; ++j) {
         const int jabs = w.j0 + j;
-        float* bias = s_bias + (x * 2 + (tile_ctr & 1)) * 128;
-        ++tile_ctr;
-        bias[rl] = next_bias;
-        if (j + 1 < n_kv) {
-          const int key = (jabs + 1) * kBN + rl;
-          next_bias = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
-        }
         ok = mbar_wait(bar(kSFull + x), s_waits++ & 1, abort_flag, p.status, kDevTimeoutAttn);
-        // one outcome for the whole warpgroup (and the bias row is visible)
+        // one outcome for the whole warpgroup
         if (named_barrier_or(1 + x, 128, !ok)) {
           ok = false;
           break;
@@ -434,55 +485,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sr[4][32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
+        if (x == 0 && j + 1 < n_kv) {
+          *aug_b_row(tile_ctr + j + 1) = aug_row(next_l);
+          fence_proxy_async_smem();  // ordered before this thread's P arrival below
+          if (j + 2 < n_kv) next_l = load_l((jabs + 2) * kBN + rl);
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
-        // t = s * scale + bias; tile max
-        // four independent max chains (short dependency chains for two warps per scheduler)
+        // tile max of S (scale > 0, so it is the max of the logits), four
+        // independent chains; on the diagonal tile key column c is visible to
+        // row rl iff c <= rl
         float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        const float4* b4 = reinterpret_cast<const float4*>(bias);
         if (jabs != it.t) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 bb = b4[(c * 32 + e) >> 2];
-              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
-                                     sc2, make_float2(bb.x, bb.y));
-              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
-                                     sc2, make_float2(bb.z, bb.w));
-              sr[c][e] = __float_as_uint(t0.x);
-              sr[c][e + 1] = __float_as_uint(t0.y);
-              sr[c][e + 2] = __float_as_uint(t1.x);
-              sr[c][e + 3] = __float_as_uint(t1.y);
-              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
-              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
-            }
+            for (int e = 0; e < 32; e += 2)
+              mxv[(c & 1) * 2 + ((e >> 1) & 1)] =
+                  max3f(mxv[(c & 1) * 2 + ((e >> 1) & 1)], __uint_as_float(sr[c][e]),
+                        __uint_as_float(sr[c][e + 1]));
           }
-        } else {  // diagonal tile: key column c is visible to row rl iff c <= rl
+        } else {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
+            for (int e = 0; e < 32; e += 2) {
               const int col = c * 32 + e;
-              const float4 bb = b4[col >> 2];
-              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
-                                     sc2, make_float2(bb.x, bb.y));
-              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
-                                     sc2, make_float2(bb.z, bb.w));
-              if (col > rl) t0.x = -INFINITY;
-              if (col + 1 > rl) t0.y = -INFINITY;
-              if (col + 2 > rl) t1.x = -INFINITY;
-              if (col + 3 > rl) t1.y = -INFINITY;
-              sr[c][e] = __float_as_uint(t0.x);
-              sr[c][e + 1] = __float_as_uint(t0.y);
-              sr[c][e + 2] = __float_as_uint(t1.x);
-              sr[c][e + 3] = __float_as_uint(t1.y);
-              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
-              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
+              if (col > rl) sr[c][e] = __float_as_uint(-INFINITY);
+              if (col + 1 > rl) sr[c][e + 1] = __float_as_uint(-INFINITY);
+              mxv[(c & 1) * 2 + ((e >> 1) & 1)] =
+                  max3f(mxv[(c & 1) * 2 + ((e >> 1) & 1)], __uint_as_float(sr[c][e]),
+                        __uint_as_float(sr[c][e + 1]));
             }
           }
         }
-        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])) * scale;
         // lazy rescale: move the reference max only when it grows by > 2^8
         float alpha = 1.0f;
         const bool grow = mx > m + kRescaleLog2;
@@ -499,8 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float2 a2 = __fadd2_rn(
-                make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), nm2);
+            const float2 a2 = __ffma2_rn(
+                make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sc2, nm2);
             const float2 p2 = make_float2(exp2_approx(a2.x), exp2_approx(a2.y));
             acc[(e >> 1) & 1] = __fadd2_rn(acc[(e >> 1) & 1], p2);
             __nv_bfloat162 pp = __floats2bfloat162_rn(p2.x, p2.y);
@@ -535,6 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(kPFull + x));
       }
       if (!ok) break;
+      tile_ctr += n_kv;
       // epilogue: O / l
       ok = mbar_wait(bar(kOFull + x), o_waits++ & 1, abort_flag, p.status, kDevTimeoutAttn);
       if (named_barrier_or(1 + x, 128, !ok)) {

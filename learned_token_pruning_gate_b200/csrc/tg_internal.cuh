@@ -269,6 +269,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// Shared-memory matrix descriptor for a K-major operand tile without swizzle:
+// element (row r, k) sits at saddr + (k / 8) * lbo + (r / 8) * sbo + (r % 8) * 16 +
+// (k % 8) * 2, i.e. 8-row x 16-byte core matrices, `lbo` bytes apart along K and
+// `sbo` bytes apart along the rows.
+__device__ __forceinline__ uint64_t nosw_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;  // descriptor version for sm_100; layout type 0 = no swizzle
+  return d;
+}
+
 // Instruction descriptor: kind::f16 with bf16 A/B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                       bool b_mn_major) {
