@@ -753,19 +753,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 // read the same K and V tiles, so each CTA stages only half of them (K: 64 of
 // the 128 keys, V: 64 of the 128 dims) and the pair's MMAs read the other half
 // from the peer: per SM, Q.K^T reads 6 KB instead of 8 KB of shared memory per
-// k-step.  With one head per CTA, TMEM holds two S buffers (2 x 128 columns)
-// next to O (128), so Q.K^T of the next tiles runs while the softmax of the
-// current one does.
+// k-step.  With one head per CTA, TMEM holds two S buffers and two output
+// accumulators (4 x 128 columns): the key tiles of a unit alternate between
+// two softmax warpgroups, each with its own S buffer, running max, row sum and
+// O, so one warpgroup's softmax overlaps the other's and the tensor core's
+// work, and no tile waits for the previous tile's softmax.  The epilogue
+// merges the two partial results (the same rule as merging key-range chunks).
 //
 //   warp 0     TMA (each CTA): its Q tile, its halves of K and V tiles into
 //              two rings; the bytes of both CTAs are counted on CTA 0's barriers
 //   warp 1     CTA 0 only: TMEM allocation for the pair and the single MMA
-//              issuer: S(0) S(1) | P(j).V_j S(j+2) | ...; commits go to the
-//              barriers of both CTAs
-//   warps 2-5  softmax of this CTA's head, one query row per thread, and the
-//              epilogue (as in the single-CTA kernel)
+//              issuer: S(0) S(1) | P(j).V_j -> O_(j mod 2), S(j+2) | ...;
+//              commits go to the barriers of both CTAs
+//   warps 2-3  idle (they complete warpgroup 0 for the register split)
+//   warps 4-7  softmax of the even key tiles of this CTA's head, warps 8-11 of
+//              the odd ones; one query row per thread.  Epilogue: the two
+//              warpgroups merge O_0 and O_1, each for half of the columns.
 // ---------------------------------------------------------------------------
-constexpr int kPairThreads = 192;
+constexpr int kPairThreads = 384;
 constexpr int kPKStages = 5, kPVStages = 5;
 
 struct PairLay {
@@ -776,8 +781,12 @@ struct PairLay {
   static constexpr uint32_t kVStage = 128 * 128;        // 128 keys x this CTA's 64 dims
   static constexpr uint32_t kK = 2 * kQBox;
   static constexpr uint32_t kV = kK + kPKStages * kKStage;
-  static constexpr uint32_t kBias = kV + kPVStages * kVStage;  // [2 parity][128] fp32
-  static constexpr uint32_t kBars = kBias + 2 * 128 * 4;
+  // bias operands of S (as in the single-CTA kernel): A (this CTA's head),
+  // B_0, B_1 (this CTA's 64 keys of the tiles in S buffer 0 / 1)
+  static constexpr uint32_t kAugTile = 4096;
+  static constexpr uint32_t kAug = kV + kPVStages * kVStage;
+  static constexpr uint32_t kML = kAug + 3 * kAugTile;  // [2 warpgroups][128] float2 (m, l)
+  static constexpr uint32_t kBars = kML + 2 * 128 * 8;
   static constexpr uint32_t kMisc = kBars + 48 * 8;
   static constexpr uint32_t kTotal = kMisc + 16;
   static constexpr uint32_t kDynSmem = kTotal + 1024;
@@ -791,8 +800,8 @@ enum {
   kPSFull = 2,     // [2 buffers], each CTA
   kPPFull = 4,     // [2 buffers], CTA 0: 256 softmax threads
   kPOFull = 6,     // each CTA
-  kPOFree = 7,     // CTA 0: 256 softmax threads
-  kPPVDone = 8,    // each CTA, one phase per P.V
+  kPOFree = 7,     // CTA 0: 512 softmax threads
+  kPAugFull = 8,   // CTA 0: 512 softmax threads, bias operands of a unit's first tiles
   kPDrain = 9,     // CTA 0
   kPKFull = 10,    // [K stages], CTA 0: both halves
   kPKEmpty = kPKFull + kPKStages,   // [K stages], each CTA
@@ -815,7 +824,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  float* s_bias = reinterpret_cast<float*>(smem + L::kBias);
+  uint8_t* s_aug = smem + L::kAug;
+  float2* s_ml = reinterpret_cast<float2*>(smem + L::kML);
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) { return smem_u32(bars + i); };
   const uint32_t rank = cluster_ctarank();
@@ -838,8 +848,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       mbar_init(bar(kPPFull + b), 256);
     }
     mbar_init(bar(kPOFull), 1);
-    mbar_init(bar(kPOFree), 256);
-    mbar_init(bar(kPPVDone), 1);
+    mbar_init(bar(kPOFree), 512);
+    mbar_init(bar(kPAugFull), 512);
     mbar_init(bar(kPDrain), 1);
     for (int s = 0; s < kPKStages; ++s) {
       mbar_init(bar(kPKFull + s), 1);
@@ -859,12 +869,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish_pair();
   }
+  // the zero halves (k = 8..15) of the bias operands are never written again
+  for (int i = threadIdx.x; i < static_cast<int>(3 * L::kAugTile / 16); i += kPairThreads)
+    reinterpret_cast<uint4*>(s_aug)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   tc_fence_before();
   cluster_sync_all();  // barriers and TMEM of both CTAs are ready
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   int q_loads = 0, k_loads = 0, v_loads = 0;  // CTA 0's TMA thread: for the abort drain
 
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
@@ -936,13 +951,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const uint64_t dq = sw128_desc(sb + L::kQ, 16, 1024);
       const uint64_t dk0 = sw128_desc(sb + L::kK, 16, 1024);
       const uint64_t dv0 = sw128_desc(sb + L::kV, L::kVStage, 1024);
-      const uint32_t t_o = tmem + 256;
+      const uint64_t d_aug_a = nosw_desc(sb + L::kAug, 2048, 128);
+      const uint64_t d_aug_b = nosw_desc(sb + L::kAug + L::kAugTile, 2048, 128);
+      // S(bf) = Q K^T + A B_bf^T (the second operand: 64 keys from each CTA)
       auto issue_s = [&](int bf, int ks) {
         const uint64_t dk = dk0 + ((ks * L::kKStage) >> 4);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk)
           umma_ss_pair(tmem + bf * 128, dq + (kk >> 2) * (L::kQBox >> 4) + (kk & 3) * 2,
                        dk + (kk >> 2) * (L::kKBox >> 4) + (kk & 3) * 2, idesc_qk, kk > 0 ? 1u : 0u);
+        umma_ss_pair(tmem + bf * 128, d_aug_a, d_aug_b + bf * (L::kAugTile >> 4), idesc_qk, 1u);
       };
       int ks = 0, vs = 0;
       uint32_t kph = 0, vph = 0;
@@ -952,6 +970,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const Unit w = decode_unit<kSplit>(p, tab, u);
         const int n_kv = w.j1 - w.j0;
         if (!wait_slot(kPQFull)) break;
+        if (!wait_slot(kPAugFull)) break;
         const int pro = n_kv < 2 ? n_kv : 2;
         for (int j = 0; j < pro; ++j) {
           if (!(ok = mbar_wait(bar(kPKFull + ks), kph, abort_flag, p.status, kDevTimeoutAttn))) break;
@@ -973,11 +992,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (!(ok = mbar_wait(bar(kPVFull + vs), vph, abort_flag, p.status, kDevTimeoutAttn))) break;
           tc_fence_after();
           const uint64_t dv = dv0 + ((vs * L::kVStage) >> 4);
+          // P(j) V_j into O_bf: the softmax warpgroup of this parity owns both
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ts_pair(t_o, tmem + bf * 128 + kk * 8, dv + kk * (2048 >> 4), idesc_pv,
-                         (j > 0 || kk > 0) ? 1u : 0u);
-          commit_both(kPPVDone);
+            umma_ts_pair(tmem + 256 + bf * 128, tmem + bf * 128 + kk * 8, dv + kk * (2048 >> 4),
+                         idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
           if (j + 1 == n_kv) commit_both(kPOFull);
           commit_both(kPVEmpty + vs);
           if (++vs == kPVStages) {
@@ -1002,14 +1021,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- softmax (warps 2-5, this CTA's head) ----------------
+    // ---------------- softmax (warps 4-11, this CTA's head) ----------------
+    if (warp < 4) {
+      // warps 2-3: no role
+    } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     const int x = static_cast<int>(rank);  // head slot within the pair
+    const int wg = (warp - 4) >> 2;       // key tiles j with j mod 2 == wg, S buffer wg, O_wg
     const int quarter = warp & 3;
     const int rl = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t t_s = tmem + lane_off;
-    const uint32_t t_o = tmem + lane_off + 256;
-    uint32_t s_ph = 0, o_waits = 0, tile_ctr = 0;
+    const uint32_t t_s = tmem + lane_off + wg * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + wg * 128;
+    uint32_t s_ph = 0, o_waits = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int u = snake_unit(round, cl, ncl);
@@ -1021,108 +1045,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const int32_t len = p.kept_start[it.b + 1] - kstart;
       const int n_kv = w.j1 - w.j0;
       const float scale = kLog2e / (sqrtf(static_cast<float>(DH)) * __ldg(p.temp + head));
-      const float gl = __ldg(p.gain + head) * kLog2e;
       const float2 sc2 = make_float2(scale, scale);
+      // bias operands: A (warpgroup 0) and this warpgroup's first B; this CTA holds
+      // keys 64 * rank .. 64 * rank + 63 of each tile, one row per thread rl < 64
+      if (wg == 0) {
+        const float cb = p.logsig ? __ldg(p.gain + head) * kLog2e / scale : 0.0f;
+        const __nv_bfloat16 c_hi = __float2bfloat16_rn(cb);
+        const __nv_bfloat16 c_lo = __float2bfloat16_rn(cb - __bfloat162float(c_hi));
+        const __nv_bfloat162 ca = __halves2bfloat162(c_hi, c_lo);
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(&ca);
+        *reinterpret_cast<uint4*>(s_aug + rl * 16) = make_uint4(cw, cw, 0u, 0u);
+      }
+      auto load_l = [&](int j) {  // log-gate of this thread's key in tile w.j0 + j
+        const int key = (w.j0 + j) * kBN + static_cast<int>(rank) * 64 + rl;
+        return (p.logsig && rl < 64 && key < len) ? __ldg(p.logsig + kstart + key) : 0.0f;
+      };
+      auto aug_row = [](float lj) {
+        lj = fmaxf(lj, -1e30f);
+        const __nv_bfloat16 l_hi = __float2bfloat16_rn(lj);
+        const __nv_bfloat16 l_lo = __float2bfloat16_rn(lj - __bfloat162float(l_hi));
+        const __nv_bfloat162 h2 = __halves2bfloat162(l_hi, l_hi), o2 = __halves2bfloat162(l_lo, l_lo);
+        return make_uint4(*reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&o2),
+                          0u, 0u);
+      };
+      uint4* b_row = reinterpret_cast<uint4*>(s_aug + (1 + wg) * L::kAugTile + rl * 16);
+      float next_l = 0.0f;
+      if (wg < n_kv && rl < 64) *b_row = aug_row(load_l(wg));
+      if (wg + 2 < n_kv) next_l = load_l(wg + 2);
+      fence_proxy_async_smem();
+      mbar_arrive_cluster(leader_bar(kPAugFull));
       float m = -INFINITY, l = 0.0f;
-      const int key0 = w.j0 * kBN + rl;
-      float next_bias = (p.logsig && key0 < len) ? gl * __ldg(p.logsig + kstart + key0) : 0.0f;
-      for (int j = 0; j < n_kv; ++j) {
+      for (int j = wg; j < n_kv; j += 2) {
         const int jabs = w.j0 + j;
-        const int bf = j & 1;
-        float* bias = s_bias + (tile_ctr & 1) * 128;
-        bias[rl] = next_bias;
-        if (j + 1 < n_kv) {
-          const int key = (jabs + 1) * kBN + rl;
-          next_bias = (p.logsig && key < len) ? gl * __ldg(p.logsig + kstart + key) : 0.0f;
-        }
-        ok = mbar_wait(bar(kPSFull + bf), (s_ph >> bf) & 1u, abort_flag, p.status, kDevTimeoutAttn);
-        s_ph ^= 1u << bf;
-        if (named_barrier_or(1, 128, !ok)) {  // one outcome for the warpgroup; bias visible
+        ok = mbar_wait(bar(kPSFull + wg), s_ph & 1u, abort_flag, p.status, kDevTimeoutAttn);
+        s_ph ^= 1u;
+        if (named_barrier_or(1 + wg, 128, !ok)) {  // one outcome for the warpgroup
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sr[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + bf * 128 + c * 32, sr[c]);
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
+        // B of tile j + 2 (same buffer): S(j) is complete, S(j + 2) waits for P(j)
+        if (j + 2 < n_kv) {
+          if (rl < 64) *b_row = aug_row(next_l);
+          fence_proxy_async_smem();
+          if (j + 4 < n_kv) next_l = load_l(j + 4);
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
         float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        const float4* b4 = reinterpret_cast<const float4*>(bias);
         if (jabs != it.t) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 bb = b4[(c * 32 + e) >> 2];
-              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
-                                     sc2, make_float2(bb.x, bb.y));
-              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
-                                     sc2, make_float2(bb.z, bb.w));
-              sr[c][e] = __float_as_uint(t0.x);
-              sr[c][e + 1] = __float_as_uint(t0.y);
-              sr[c][e + 2] = __float_as_uint(t1.x);
-              sr[c][e + 3] = __float_as_uint(t1.y);
-              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
-              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
-            }
+            for (int e = 0; e < 32; e += 2)
+              mxv[(c & 1) * 2 + ((e >> 1) & 1)] =
+                  max3f(mxv[(c & 1) * 2 + ((e >> 1) & 1)], __uint_as_float(sr[c][e]),
+                        __uint_as_float(sr[c][e + 1]));
           }
         } else {  // diagonal tile: key column c is visible to row rl iff c <= rl
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
+            for (int e = 0; e < 32; e += 2) {
               const int col = c * 32 + e;
-              const float4 bb = b4[col >> 2];
-              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
-                                     sc2, make_float2(bb.x, bb.y));
-              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])),
-                                     sc2, make_float2(bb.z, bb.w));
-              if (col > rl) t0.x = -INFINITY;
-              if (col + 1 > rl) t0.y = -INFINITY;
-              if (col + 2 > rl) t1.x = -INFINITY;
-              if (col + 3 > rl) t1.y = -INFINITY;
-              sr[c][e] = __float_as_uint(t0.x);
-              sr[c][e + 1] = __float_as_uint(t0.y);
-              sr[c][e + 2] = __float_as_uint(t1.x);
-              sr[c][e + 3] = __float_as_uint(t1.y);
-              mxv[(c & 1) * 2] = max3f(mxv[(c & 1) * 2], t0.x, t0.y);
-              mxv[(c & 1) * 2 + 1] = max3f(mxv[(c & 1) * 2 + 1], t1.x, t1.y);
+              if (col > rl) sr[c][e] = __float_as_uint(-INFINITY);
+              if (col + 1 > rl) sr[c][e + 1] = __float_as_uint(-INFINITY);
+              mxv[(c & 1) * 2 + ((e >> 1) & 1)] =
+                  max3f(mxv[(c & 1) * 2 + ((e >> 1) & 1)], __uint_as_float(sr[c][e]),
+                        __uint_as_float(sr[c][e + 1]));
             }
           }
         }
-        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])) * scale;
         float alpha = 1.0f;
         const bool grow = mx > m + kRescaleLog2;
         if (grow) {
           alpha = exp2_approx(m - mx);
           m = mx;
         }
-        // O holds this unit's earlier P.V; rescaling it needs the last one done
-        // (warp-uniform: tcgen05.ld/st are collective)
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          if (!mbar_wait(bar(kPPVDone), (tile_ctr - 1) & 1, abort_flag, p.status, kDevTimeoutAttn))
-            ok = false;
-          tc_fence_after();
-          if (ok) {
-#pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {
-              uint32_t orow[32];
-              tmem_ld32(t_o + c * 32, orow);
-              tmem_ld_wait(orow);
-#pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                const float2 v2 = __fmul2_rn(
-                    make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
-                    make_float2(alpha, alpha));
-                orow[e] = __float_as_uint(v2.x);
-                orow[e + 1] = __float_as_uint(v2.y);
-              }
-              tmem_st32(t_o + c * 32, orow);
-            }
-          }
-        }
-        ++tile_ctr;
         const float2 nm2 = make_float2(-m, -m);
         float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
@@ -1130,44 +1133,84 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float2 a2 = __fadd2_rn(
-                make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), nm2);
+            const float2 a2 = __ffma2_rn(
+                make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sc2, nm2);
             const float2 p2 = make_float2(exp2_approx(a2.x), exp2_approx(a2.y));
             acc[(e >> 1) & 1] = __fadd2_rn(acc[(e >> 1) & 1], p2);
             __nv_bfloat162 pp = __floats2bfloat162_rn(p2.x, p2.y);
             pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
           }
-          tmem_st16(t_s + bf * 128 + c * 16, pk);
+          tmem_st16(t_s + c * 16, pk);
         }
         l = fmaf(l, alpha, (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
+        // O_wg holds P.V of this warpgroup's earlier tiles; the last of them was
+        // issued before S(j), which is complete, and P(j).V is not issued before
+        // P is marked full: O_wg may be rescaled in place (warp-uniform)
+        if (j > wg && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t orow[32];
+            tmem_ld32(t_o + c * 32, orow);
+            tmem_ld_wait(orow);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v2 = __fmul2_rn(
+                  make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
+                  make_float2(alpha, alpha));
+              orow[e] = __float_as_uint(v2.x);
+              orow[e + 1] = __float_as_uint(v2.y);
+            }
+            tmem_st32(t_o + c * 32, orow);
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive_cluster(leader_bar(kPPFull + bf));
+        mbar_arrive_cluster(leader_bar(kPPFull + wg));
       }
-      if (named_barrier_or(1, 128, !ok)) {  // a rescale wait may have failed on the last tile
-        ok = false;
-        break;
-      }
-      ok = mbar_wait(bar(kPOFull), o_waits++ & 1, abort_flag, p.status, kDevTimeoutAttn);
-      if (named_barrier_or(1, 128, !ok)) {
+      // both warpgroups take the same way out of the unit
+      if (named_barrier_or(1 + wg, 128, !ok)) ok = false;
+      if (ok) ok = mbar_wait(bar(kPOFull), o_waits++ & 1, abort_flag, p.status, kDevTimeoutAttn);
+      s_ml[wg * 128 + rl] = make_float2(m, l);
+      if (named_barrier_or(3, 256, !ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      // merge: O = (2^(m0-M) O_0 + 2^(m1-M) O_1) / (2^(m0-M) l_0 + 2^(m1-M) l_1);
+      // warpgroup 0 writes columns 0-63, warpgroup 1 columns 64-127
+      const float2 ml0 = s_ml[rl], ml1 = s_ml[128 + rl];
+      const bool two = n_kv > 1;
+      const float mm = two ? fmaxf(ml0.x, ml1.x) : ml0.x;
+      const float f0 = exp2f(ml0.x - mm), f1 = two ? exp2f(ml1.x - mm) : 0.0f;
+      const float lsum = f0 * ml0.y + f1 * ml1.y;
+      const float inv = 1.0f / lsum;
+      const float g0 = f0 * inv, g1 = f1 * inv;
       const int qi = it.t * kBM + rl;
-      const float inv = 1.0f / l;
       __nv_bfloat16* out = p.out + (static_cast<int64_t>(kstart + qi) * p.hq + head) * DH;
+      const uint32_t t_o0 = tmem + lane_off + 256, t_o1 = tmem + lane_off + 384;
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
-        uint32_t orow[32];
-        tmem_ld32(t_o + c * 32, orow);
-        tmem_ld_wait(orow);
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = wg * 2 + cc;
+        uint32_t o0[32], o1[32];
+        tmem_ld32(t_o0 + c * 32, o0);
+        if (two) tmem_ld32(t_o1 + c * 32, o1);
+        tmem_ld_wait(o0);
+        if (two) {
+          tmem_ld_wait(o1);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o1[e] = 0u;
+        }
         if (qi < len) {
           uint32_t pkd[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(orow[2 * e]) * inv,
-                                                      __uint_as_float(orow[2 * e + 1]) * inv);
+            const float v0 = two ? fmaf(__uint_as_float(o0[2 * e]), g0, __uint_as_float(o1[2 * e]) * g1)
+                                 : __uint_as_float(o0[2 * e]) * g0;
+            const float v1 = two ? fmaf(__uint_as_float(o0[2 * e + 1]), g0,
+                                        __uint_as_float(o1[2 * e + 1]) * g1)
+                                 : __uint_as_float(o0[2 * e + 1]) * g0;
+            __nv_bfloat162 pp = __floats2bfloat162_rn(v0, v1);
             pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
           }
           uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
@@ -1178,8 +1221,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
       tc_fence_before();
       mbar_arrive_cluster(leader_bar(kPOFree));
-      if (p.lse && qi < len)
-        p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (m + log2f(l)) * kLn2;
+      if (wg == 0 && p.lse && qi < len)
+        p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (mm + log2f(lsum)) * kLn2;
+    }
     }
   }
 
@@ -1429,7 +1473,7 @@ tg_status launch_pair(const void* q, const void* k, const void* v, const TcParam
 // each (a unit then runs on two SMs); the single-CTA kernel, two softmax
 // warpgroups per SM, has the higher throughput per SM.  The modelled
 // makespans of the two plans decide.
-constexpr double kTilePair = 0.72;  // pair kernel's tile time, in single-CTA tile times
+constexpr double kTilePair = 0.55;  // pair kernel's tile time, in single-CTA tile times
 constexpr double kMergeCost = 3.0;
 static bool pairs_possible(const TcParams& p, int hkv, int dh) {
   return dh == 128 && (p.hq / hkv) % 2 == 0 && num_sms() >= 2 && p.n_items <= num_sms();

@@ -173,8 +173,10 @@ def test_attention_workspace_plan(L):
 
     if torch.cuda.is_available():
         pytest.skip("plan sizes below assume 148 SMs")
-    st, b = _ws_bytes(L, [0, 1280])  # one 32k-token prompt kept down to 1280 rows
+    st, b = _ws_bytes(L, [0, 1280], hq=12, hkv=4)  # one prompt kept down to 1280 rows
     assert st == 0 and b > 0
+    # with even GQA groups the same batch runs on CTA pairs, which never split
+    assert _ws_bytes(L, [0, 1280]) == (0, 0)
     # every partial slot holds 2 heads x 128 rows x (head_dim + 1) floats, plus counters
     assert b % 4 == 0 and b >= 2 * 128 * 129 * 4
     st, b = _ws_bytes(L, [0, 8448])  # 66 query tiles x 8 head pairs: no split
@@ -187,10 +189,10 @@ def test_attention_workspace_plan(L):
     _, ck = _arr([0, 10])
     assert L.tg_attention_workspace_bytes(0, 1, ck, 16, 8, 128, 0, None) == INVALID
     # a workspace smaller than the plan needs is refused before anything launches
-    st, need = _ws_bytes(L, [0, 1280])
+    st, need = _ws_bytes(L, [0, 1280], hq=12, hkv=4)
     _, ck = _arr([0, 1280])
     a = L.tg_gated_attention
-    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 16, 8, 128, None, FAKE, FAKE, FAKE, None, FAKE,
+    assert a(FAKE, FAKE, FAKE, 0, 1, ck, 12, 4, 128, None, FAKE, FAKE, FAKE, None, FAKE,
              need - 16, 0, None) == WORKSPACE
     assert b"needed" in L.tg_last_error_message()
 
@@ -203,8 +205,9 @@ def test_attention_kernel_choice():
     if torch.cuda.is_available():
         pytest.skip("choices below assume 148 SMs")
     assert tg.attention_kernel([0, 2304], 16, 8, 128) == "attn_pair_kernel"
-    assert tg.attention_kernel([0, 1280], 16, 8, 128) == "attn_tc_kernel (key-range split)"
-    assert tg.attention_kernel([0, 1280], 16, 8, 128, with_workspace=False) == "attn_pair_kernel"
+    assert tg.attention_kernel([0, 1280], 16, 8, 128) == "attn_pair_kernel"
+    assert tg.attention_kernel([0, 1280], 12, 4, 128) == "attn_tc_kernel (key-range split)"
+    assert tg.attention_kernel([0, 1280], 12, 4, 128, with_workspace=False) == "attn_tc_kernel"
     assert tg.attention_kernel([0, 8448], 16, 8, 128) == "attn_tc_kernel"
     assert tg.attention_kernel([0, 2304], 12, 4, 128, with_workspace=False) == "attn_tc_kernel"
     assert tg.attention_kernel([0, 2304], 16, 8, 64, with_workspace=False) == "attn_tc_kernel"

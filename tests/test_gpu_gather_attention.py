@@ -94,7 +94,7 @@ def test_attention_without_workspace(oracle, lens):
                workspace=None)
 
 
-@pytest.mark.parametrize("lens,Hq,Hkv,dh", [([1000], 16, 8, 128), ([1280], 16, 8, 128),
+@pytest.mark.parametrize("lens,Hq,Hkv,dh", [([1000], 16, 8, 64), ([1280], 12, 4, 128),
                                             ([700, 90, 1500], 12, 4, 128), ([900], 4, 2, 64)])
 def test_attention_split_matches_unsplit_and_repeats(lens, Hq, Hkv, dh):
     """Small batches split long query tiles over several SMs; the merged result

@@ -29,11 +29,12 @@ def _noalloc(q, k, v, cu, ls, gain, temp, out, lse):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("lens", [[1000], [2304], [5, 0, 260, 1, 640], [8448]])
-def test_noalloc_matches_workspace_call_twice(lens):
+@pytest.mark.parametrize("lens,Hq,Hkv", [([1000], 16, 8), ([2304], 16, 8), ([5, 0, 260, 1, 640], 16, 8),
+                                         ([8448], 16, 8), ([1280], 12, 4), ([2304], 12, 4)])
+def test_noalloc_matches_workspace_call_twice(lens, Hq, Hkv):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    Hq, Hkv, dh = 16, 8, 128
+    dh = 128
     cu, q, k, v, ls, gain, temp = gen.attention_inputs(lens, Hq, Hkv, dh, 31 + len(lens), "bf16",
                                                        True)
     q, k, v, ls, gain, temp = (dev(x) for x in (q, k, v, ls, gain, temp))
