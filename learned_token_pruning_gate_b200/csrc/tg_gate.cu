@@ -23,6 +23,43 @@ __device__ __forceinline__ float gelu_erf(float a) {
   return 0.5f * a * (1.0f + erff(a * 0.70710678118654752f));
 }
 
+// GELU for the tensor-core epilogues: GELU(a) = a Phi(a), Phi(a) = (1 + erf(a/sqrt2)) / 2,
+// with erf from the rational-exponential approximation of Abramowitz & Stegun
+// (Handbook of Mathematical Functions, 7.1.26, after C. Hastings): for x >= 0,
+//   1 - erf(x) = t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) e^(-x^2),  t = 1 / (1 + p x),
+// absolute error <= 1.5e-7.  With h = a (1 - erf(|a|/sqrt2)) / 2, GELU(a) is a - h for
+// a >= 0 and h for a < 0.  One reciprocal and one exponential on the special-function
+// unit, seven FMA-pipe operations.
+__device__ __forceinline__ float gelu_as(float a) {
+  const float x = fabsf(a) * 0.70710678118654752f;
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, x, 1.0f)));
+  float q = fmaf(t, 1.061405429f, -1.453152027f);
+  q = fmaf(q, t, 1.421413741f);
+  q = fmaf(q, t, -0.284496736f);
+  q = fmaf(q, t, 0.254829592f);
+  q *= t;
+  const float e = exp2_approx(-1.4426950408889634f * x * x);
+  const float h = 0.5f * a * (q * e);
+  return a >= 0.0f ? a - h : h;
+}
+// w2 . GELU(acc + b1) over 32 accumulator columns (b1, w2 in shared memory,
+// 16-byte aligned), two partial sums
+__device__ __forceinline__ float gelu_dot32(const uint32_t (&r)[32], const float* b1, const float* w2,
+                                            float sum) {
+  float s2 = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float4 bb = *reinterpret_cast<const float4*>(b1 + j);
+    const float4 ww = *reinterpret_cast<const float4*>(w2 + j);
+    sum = fmaf(ww.x, gelu_as(__uint_as_float(r[j]) + bb.x), sum);
+    s2 = fmaf(ww.y, gelu_as(__uint_as_float(r[j + 1]) + bb.y), s2);
+    sum = fmaf(ww.z, gelu_as(__uint_as_float(r[j + 2]) + bb.z), sum);
+    s2 = fmaf(ww.w, gelu_as(__uint_as_float(r[j + 3]) + bb.w), s2);
+  }
+  return sum + s2;
+}
+
 template <typename T>
 __device__ __forceinline__ float to_f(T x);
 template <>
@@ -207,9 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld32(t_addr + c, r);
         tmem_ld_wait(r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          sum = fmaf(s_w2[c + j], gelu_erf(__uint_as_float(r[j]) + s_b1[c + j]), sum);
+        sum = gelu_dot32(r, s_b1 + c, s_w2 + c, sum);
       }
       tc_fence_before();
       mbar_arrive(bar(10 + acc));
@@ -300,12 +335,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish_pair();
   }
-  if (warp >= 2) {
-    for (int i = threadIdx.x - 64; i < p.dg; i += 256) {
-      s_b1[i] = p.b1[i];
-      s_w2[i] = p.w2[i];
-    }
-  }
   tc_fence_before();
   cluster_sync_all();  // barriers and TMEM of both CTAs are ready
   tc_fence_after();
@@ -383,6 +412,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     const int c_split = ((p.dg / 32) / 2) * 32;
     const int c_lo = half ? c_split : 0, c_hi = half ? p.dg : c_split;
     float* s_part = reinterpret_cast<float*>(smem + L.part_off);
+    // b1 and w2 into shared memory while the first tile's MMAs run
+    for (int i = threadIdx.x - 64; i < p.dg; i += 256) {
+      s_b1[i] = p.b1[i];
+      s_w2[i] = p.w2[i];
+    }
+    named_barrier(2, 256);
     uint32_t acc = 0, acc_phase = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs) {
       if (!mbar_wait(bar(12 + acc), acc_phase, abort_flag, p.status, kDevTimeoutGate)) break;
@@ -394,9 +429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         uint32_t r[32];
         tmem_ld32(t_addr + c, r);
         tmem_ld_wait(r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          sum = fmaf(s_w2[c + j], gelu_erf(__uint_as_float(r[j]) + s_b1[c + j]), sum);
+        sum = gelu_dot32(r, s_b1 + c, s_w2 + c, sum);
       }
       tc_fence_before();
       mbar_arrive_cluster(leader_bar(14 + acc));
