@@ -259,6 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_dep_wait();  // q', k', v' and the log-gates are complete
+  grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
 
   int q_loads = 0, tiles_loaded = 0;  // producer thread: loads issued (for the abort drain)
@@ -876,6 +878,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   tc_fence_before();
   cluster_sync_all();  // barriers and TMEM of both CTAs are ready
   tc_fence_after();
+  grid_dep_wait();  // q', k', v' and the log-gates are complete
+  grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
   int q_loads = 0, k_loads = 0, v_loads = 0;  // CTA 0's TMA thread: for the abort drain
 
@@ -1443,8 +1447,13 @@ tg_status launch_dh(const void* q, const void* k, const void* v, const TcParams&
                                                 static_cast<int>(Ly::kDynSmem)),
                            "attn smem attribute");
   if (r != TG_OK) return r;
-  attn_tc_kernel<DH, kSplit><<<grid, kThreads, Ly::kDynSmem, st>>>(tq, tk, tv, p, tab);
-  return cuda_check(cudaGetLastError(), "attn_tc launch");
+  if (kSplit) {  // the counter reset runs just before: plain stream order
+    attn_tc_kernel<DH, kSplit><<<grid, kThreads, Ly::kDynSmem, st>>>(tq, tk, tv, p, tab);
+    return cuda_check(cudaGetLastError(), "attn_tc launch");
+  }
+  return cuda_check(launch_pdl(attn_tc_kernel<DH, kSplit>, dim3(grid), dim3(kThreads), Ly::kDynSmem,
+                               st, tq, tk, tv, p, tab),
+                    "attn_tc launch");
 }
 
 tg_status launch_pair(const void* q, const void* k, const void* v, const TcParams& p, int clusters,
@@ -1464,8 +1473,9 @@ tg_status launch_pair(const void* q, const void* k, const void* v, const TcParam
                                                 static_cast<int>(PairLay::kDynSmem)),
                            "attn pair smem attribute");
   if (r != TG_OK) return r;
-  attn_pair_kernel<<<2 * clusters, kPairThreads, PairLay::kDynSmem, st>>>(tq, tk, tv, p);
-  return cuda_check(cudaGetLastError(), "attn_pair launch");
+  return cuda_check(launch_pdl(attn_pair_kernel, dim3(2 * clusters), dim3(kPairThreads),
+                               PairLay::kDynSmem, st, tq, tk, tv, p),
+                    "attn_pair launch");
 }
 
 // CTA pairs need an even group (both heads of every pair exist) and head_dim 128.

@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(256) gate_simt_kernel(const T* __restrict__ h,
                                                         const float* __restrict__ w2, float b2,
                                                         float* __restrict__ z) {
   const int lane = threadIdx.x & 31;
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t j = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        j < n; j += warps) {
@@ -171,6 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_dep_wait();  // (launched in stream order: returns at once)
+  grid_dep_launch();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
@@ -338,6 +342,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   tc_fence_before();
   cluster_sync_all();  // barriers and TMEM of both CTAs are ready
   tc_fence_after();
+  grid_dep_wait();  // (launched in stream order: returns at once)
+  grid_dep_launch();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {

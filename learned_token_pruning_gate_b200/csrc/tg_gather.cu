@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(kWarps * 32) gather_kernel(const __grid_consta
   __shared__ float s_sin[kWarps][kMaxHalf];
 
   const int B = p.pt.batch;
+  grid_dep_wait();  // the kept indices and scores are complete
+  grid_dep_launch();
   for (int i = threadIdx.x; i <= B; i += blockDim.x) {
     s_kept_start[i] = p.pt.kept_start[i];
     s_start[i] = p.pt.start[i];
@@ -272,6 +274,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) gather_bulk_kernel(const __gr
     sm.kept_start[i] = p.pt.kept_start[i];
     sm.start[i] = p.pt.start[i];
   }
+  grid_dep_wait();  // the kept indices and scores are complete
+  grid_dep_launch();
   // this CTA's kept indices (batches blockIdx.x, blockIdx.x + G, ...), so the
   // load thread never waits on an index; batches past the buffer read theirs
   // one batch ahead instead
@@ -550,27 +554,30 @@ tg_status launch_gather(const int32_t* kept_idx, int64_t m_total, const PromptTa
                                             static_cast<int>(smem)),
                        "gather smem attribute");
         if (r != TG_OK) return r;
-        gather_bulk_kernel<__nv_bfloat16><<<grid, kBulkThreads, smem, st>>>(b);
+        r = cuda_check(launch_pdl(gather_bulk_kernel<__nv_bfloat16>, dim3(grid), dim3(kBulkThreads),
+                                  smem, st, b),
+                       "gather launch");
       } else {
         r = cuda_check(cudaFuncSetAttribute(gather_bulk_kernel<float>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             static_cast<int>(smem)),
                        "gather smem attribute");
         if (r != TG_OK) return r;
-        gather_bulk_kernel<float><<<grid, kBulkThreads, smem, st>>>(b);
+        r = cuda_check(launch_pdl(gather_bulk_kernel<float>, dim3(grid), dim3(kBulkThreads), smem,
+                                  st, b),
+                       "gather launch");
       }
-      return cuda_check(cudaGetLastError(), "gather launch");
+      return r;
     }
   }
   const int64_t items = m_total * nt;
   int64_t blocks = (items + kWarps - 1) / kWarps;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
   if (blocks > cap) blocks = cap;
+  const dim3 g(static_cast<unsigned>(blocks)), blk(kWarps * 32);
   if (dt == TG_BF16)
-    gather_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kWarps * 32, 0, st>>>(p);
-  else
-    gather_kernel<float><<<static_cast<unsigned>(blocks), kWarps * 32, 0, st>>>(p);
-  return cuda_check(cudaGetLastError(), "gather launch");
+    return cuda_check(launch_pdl(gather_kernel<__nv_bfloat16>, g, blk, 0, st, p), "gather launch");
+  return cuda_check(launch_pdl(gather_kernel<float>, g, blk, 0, st, p), "gather launch");
 }
 
 }  // namespace tg

@@ -424,10 +424,40 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl() may start
+// while the previous kernel in its stream is still running.  grid_dep_wait()
+// returns once that kernel has completed and its writes are visible (at once
+// when the kernel was launched without the attribute); a kernel reads nothing
+// that earlier work in the stream writes, and writes nothing, before it.
+// grid_dep_launch() lets the next kernel of the stream start; every kernel
+// calls it only after its own grid_dep_wait(), so when a kernel starts, all
+// work before its predecessor is complete.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float exp2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Host: launch with programmatic dependent launch allowed (see grid_dep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 #endif  // __CUDACC__

@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
     s_total[1][i] = 0;
   }
   __syncthreads();
+  grid_dep_wait();  // the scores are complete
+  grid_dep_launch();
   // keys into shared memory; pass-0 histogram (top 11 bits) on the way
   for (int i = tid; i < len; i += kThreads) {
     const uint32_t key =
@@ -287,13 +289,15 @@ tg_status launch_topk(const float* z, const uint32_t* keys, const PromptTable* t
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = dyn;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cl;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see grid_dep_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cuda_check(cudaLaunchKernelEx(&cfg, kernel, p), "topk launch");
 }
 
