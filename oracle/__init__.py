@@ -62,8 +62,15 @@ def _load():
                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                           _f32p, _f32p, _f32p, _i64p, ctypes.c_int64, _f64p,
                                           _f64p]
+        L.tgo_attention_loss.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int32, _i32p, ctypes.c_int32,
+                                         ctypes.c_int32, ctypes.c_int32, _f64p, _f64p, _f64p, _f32p,
+                                         _f64p]
+        L.tgo_gated_attention_backward.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int32, _i32p,
+                                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                   _f64p, _f64p, _f64p, _f32p, _f64p, _f64p, _f64p]
         for name in ("tgo_gate_score", "tgo_topk_select", "tgo_select_by_keys",
-                     "tgo_gather_rows", "tgo_logsig", "tgo_gated_attention"):
+                     "tgo_gather_rows", "tgo_logsig", "tgo_gated_attention", "tgo_attention_loss",
+                     "tgo_gated_attention_backward"):
             getattr(L, name).restype = ctypes.c_int
     return _lib
 
@@ -204,3 +211,46 @@ def gated_attention(q, k, v, cu_kept, logsig=None, gain=None, temp=None, rows=No
                                  _p(temp, _f32p), _p(r, _i64p), cnt, _p(out, _f64p),
                                  _p(lse, _f64p)), "gated_attention")
     return out, lse
+
+
+def _bwd_args(q, k, v, cu_kept, logsig, gain, temp, dout):
+    q = _c(q, np.float32)
+    k = _c(k, np.float32)
+    v = _c(v, np.float32)
+    dout = _c(dout, np.float32)
+    cu = _c(cu_kept, np.int32)
+    ls = _c(logsig, np.float64)
+    g = _c(gain, np.float64)
+    t = _c(temp, np.float64)
+    M, Hq, dh = q.shape
+    assert dout.shape == q.shape and ls.shape == (M,) and g.shape == (Hq,) and t.shape == (Hq,)
+    return q, k, v, dout, cu, ls, g, t, Hq, k.shape[1], dh
+
+
+def attention_loss(q, k, v, cu_kept, logsig, gain, temp, dout) -> float:
+    """L = sum(dout * out) of the gated attention in fp64 (double log-gates, gains
+    and temperatures), the scalar whose gradient gated_attention_backward gives."""
+    L = _load()
+    q, k, v, dout, cu, ls, g, t, Hq, Hkv, dh = _bwd_args(q, k, v, cu_kept, logsig, gain, temp, dout)
+    out = np.zeros(1, np.float64)
+    _check(L.tgo_attention_loss(_p(q, _f32p), _p(k, _f32p), _p(v, _f32p), cu.shape[0] - 1,
+                                _p(cu, _i32p), Hq, Hkv, dh, _p(ls, _f64p), _p(g, _f64p),
+                                _p(t, _f64p), _p(dout, _f32p), _p(out, _f64p)), "attention_loss")
+    return float(out[0])
+
+
+def gated_attention_backward(q, k, v, cu_kept, logsig, gain, temp, dout):
+    """Exact fp64 gradient of sum(dout * out) with respect to the log-gates l
+    [M], the gains g [Hq] and the temperatures tau [Hq]."""
+    L = _load()
+    q, k, v, dout, cu, ls, g, t, Hq, Hkv, dh = _bwd_args(q, k, v, cu_kept, logsig, gain, temp, dout)
+    M = q.shape[0]
+    d_l = np.zeros(max(M, 1), np.float64)
+    d_g = np.zeros(Hq, np.float64)
+    d_t = np.zeros(Hq, np.float64)
+    _check(L.tgo_gated_attention_backward(_p(q, _f32p), _p(k, _f32p), _p(v, _f32p),
+                                          cu.shape[0] - 1, _p(cu, _i32p), Hq, Hkv, dh,
+                                          _p(ls, _f64p), _p(g, _f64p), _p(t, _f64p),
+                                          _p(dout, _f32p), _p(d_l, _f64p), _p(d_g, _f64p),
+                                          _p(d_t, _f64p)), "gated_attention_backward")
+    return d_l[:M], d_g, d_t

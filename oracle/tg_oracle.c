@@ -352,3 +352,150 @@ int tgo_gated_attention(const float* q, const float* k, const float* v, int32_t 
     }
     return 0;
 }
+
+/* ---- backward of the gated attention --------------------------------------
+ *
+ * The gate is trained through the attention bias (pages: the gate's scores
+ * enter the attention logits above the gate as a bias, the "MoE router trick",
+ * which is what carries a gradient back to the scorer).  For a scalar loss
+ * L = sum over rows i, heads h, dims c of dout[i,h,c] * out[i,h,c] these
+ * functions give L itself and its exact gradient with respect to the kept
+ * rows' log-gates l_j, the per-head gains g_h and temperatures tau_h, all in
+ * fp64 from double parameters (so that finite differences can check them).
+ *
+ * Per prompt, head h and query row i (keys j <= i of the same prompt):
+ *   logit_ij = (q_i . k_j) / (sqrt(d_h) tau_h) + g_h l_j,  P_ij = softmax_j(logit_ij)
+ *   dP_ij = dout_i . v_j,   D_i = sum_j P_ij dP_ij,   dlogit_ij = P_ij (dP_ij - D_i)
+ *   dL/dl_j  += g_h dlogit_ij
+ *   dL/dg_h  += l_j dlogit_ij
+ *   dL/dtau_h += dlogit_ij * (-(q_i . k_j) / (sqrt(d_h) tau_h^2))
+ * (the derivative of the softmax-weighted sum out_i = sum_j P_ij v_j through
+ * the logits; D_i equals dout_i . out_i).
+ */
+static void attn_row_f64(const float* q, const float* k, int64_t i, int64_t j0,
+                         int32_t h, int32_t hk, int32_t Hq, int32_t Hkv, int32_t dh,
+                         const double* logsig, const double* gain, const double* temp,
+                         double* s, double* P) {
+    const float* qi = q + (i * Hq + h) * (int64_t)dh;
+    double scale = 1.0 / (sqrt((double)dh) * temp[h]);
+    double mx = -INFINITY;
+    for (int64_t j = j0; j <= i; ++j) {
+        const float* kj = k + (j * Hkv + hk) * (int64_t)dh;
+        double dot = 0.0;
+        for (int32_t c = 0; c < dh; ++c) dot += (double)qi[c] * (double)kj[c];
+        s[j - j0] = dot;
+        double lg = dot * scale + gain[h] * logsig[j];
+        P[j - j0] = lg;
+        if (lg > mx) mx = lg;
+    }
+    double denom = 0.0;
+    for (int64_t j = j0; j <= i; ++j) {
+        P[j - j0] = exp(P[j - j0] - mx);
+        denom += P[j - j0];
+    }
+    for (int64_t j = j0; j <= i; ++j) P[j - j0] /= denom;
+}
+
+static int32_t prompt_of(const int32_t* cu, int32_t B, int64_t i) {
+    int32_t b = 0;
+    while (b + 1 < B && cu[b + 1] <= i) ++b;
+    return b;
+}
+
+int tgo_attention_loss(const float* q, const float* k, const float* v, int32_t B,
+                       const int32_t* cu_kept, int32_t Hq, int32_t Hkv, int32_t dh,
+                       const double* logsig, const double* gain, const double* temp,
+                       const float* dout, double* loss_out) {
+    if (!q || !k || !v || !cu_kept || !logsig || !gain || !temp || !dout || !loss_out) return 1;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || dh <= 0) return 1;
+    int64_t M = cu_kept[B];
+    int32_t group = Hq / Hkv;
+    double total = 0.0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : total)
+    for (int64_t i = 0; i < M; ++i) {
+        int64_t j0 = cu_kept[prompt_of(cu_kept, B, i)];
+        int64_t nk = i - j0 + 1;
+        double* s = (double*)malloc(sizeof(double) * (size_t)nk);
+        double* P = (double*)malloc(sizeof(double) * (size_t)nk);
+        for (int32_t h = 0; h < Hq; ++h) {
+            int32_t hk = h / group;
+            attn_row_f64(q, k, i, j0, h, hk, Hq, Hkv, dh, logsig, gain, temp, s, P);
+            const float* di = dout + (i * Hq + h) * (int64_t)dh;
+            for (int64_t j = j0; j <= i; ++j) {
+                const float* vj = v + (j * Hkv + hk) * (int64_t)dh;
+                double dp = 0.0;
+                for (int32_t c = 0; c < dh; ++c) dp += (double)di[c] * (double)vj[c];
+                total += P[j - j0] * dp;
+            }
+        }
+        free(s);
+        free(P);
+    }
+    *loss_out = total;
+    return 0;
+}
+
+int tgo_gated_attention_backward(const float* q, const float* k, const float* v, int32_t B,
+                                 const int32_t* cu_kept, int32_t Hq, int32_t Hkv, int32_t dh,
+                                 const double* logsig, const double* gain, const double* temp,
+                                 const float* dout, double* d_logsig, double* d_gain,
+                                 double* d_temp) {
+    if (!q || !k || !v || !cu_kept || !logsig || !gain || !temp || !dout || !d_logsig || !d_gain ||
+        !d_temp)
+        return 1;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || dh <= 0) return 1;
+    int64_t M = cu_kept[B];
+    int32_t group = Hq / Hkv;
+    for (int64_t j = 0; j < M; ++j) d_logsig[j] = 0.0;
+    for (int32_t h = 0; h < Hq; ++h) d_gain[h] = d_temp[h] = 0.0;
+#pragma omp parallel
+    {
+        /* each thread sums into its own buffers; they are added up at the end */
+        double* dl = (double*)calloc((size_t)(M > 0 ? M : 1), sizeof(double));
+        double* dg = (double*)calloc((size_t)Hq, sizeof(double));
+        double* dtau = (double*)calloc((size_t)Hq, sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < M; ++i) {
+            int64_t j0 = cu_kept[prompt_of(cu_kept, B, i)];
+            int64_t nk = i - j0 + 1;
+            double* s = (double*)malloc(sizeof(double) * (size_t)nk);
+            double* P = (double*)malloc(sizeof(double) * (size_t)nk);
+            double* dP = (double*)malloc(sizeof(double) * (size_t)nk);
+            for (int32_t h = 0; h < Hq; ++h) {
+                int32_t hk = h / group;
+                attn_row_f64(q, k, i, j0, h, hk, Hq, Hkv, dh, logsig, gain, temp, s, P);
+                const float* di = dout + (i * Hq + h) * (int64_t)dh;
+                double D = 0.0;
+                for (int64_t j = j0; j <= i; ++j) {
+                    const float* vj = v + (j * Hkv + hk) * (int64_t)dh;
+                    double dp = 0.0;
+                    for (int32_t c = 0; c < dh; ++c) dp += (double)di[c] * (double)vj[c];
+                    dP[j - j0] = dp;
+                    D += P[j - j0] * dp;
+                }
+                double scale = 1.0 / (sqrt((double)dh) * temp[h]);
+                for (int64_t j = j0; j <= i; ++j) {
+                    double dlogit = P[j - j0] * (dP[j - j0] - D);
+                    dl[j] += gain[h] * dlogit;
+                    dg[h] += logsig[j] * dlogit;
+                    dtau[h] += dlogit * (-s[j - j0] * scale / temp[h]);
+                }
+            }
+            free(s);
+            free(P);
+            free(dP);
+        }
+#pragma omp critical
+        {
+            for (int64_t j = 0; j < M; ++j) d_logsig[j] += dl[j];
+            for (int32_t h = 0; h < Hq; ++h) {
+                d_gain[h] += dg[h];
+                d_temp[h] += dtau[h];
+            }
+        }
+        free(dl);
+        free(dg);
+        free(dtau);
+    }
+    return 0;
+}
