@@ -287,6 +287,50 @@ TG_API tg_status tg_gated_attention_noalloc(const void* q, const void* k, const 
                                      const float* gain, const float* temp, void* out, float* lse,
                                      int32_t algo, tg_stream_t stream);
 
+/*
+ * Backward of tg_gated_attention: the gradient that trains the gate.  The
+ * gate's score enters every attention layer above the gate as a bias on the
+ * logits scaled by a per-head gain (TokenGate, "How it works": the Mixture-of-
+ * Experts router trick), so a loss on the attention output reaches the scorer
+ * through it; the per-head gains and temperatures are learned the same way.
+ *
+ * For a scalar loss L and dout = dL/dout [M, Hq, head_dim] (dtype of q), with
+ * out and lse the forward's outputs for the same inputs, the call writes (fp32,
+ * overwritten, device):
+ *   d_logsig [M]  dL/dl_j for every kept row j (l = logsig, the bias input)
+ *   d_z_kept [M]  dL/dz of the kept rows' gate scores, d_logsig * (1 - exp(l)):
+ *                 l = log sigmoid(z) for document rows; question rows (l fixed
+ *                 at 0) get 0
+ *   d_gain [Hq]   dL/dg_h
+ *   d_temp [Hq]   dL/dtau_h
+ * Per prompt, head h and query row i, with P the attention weights,
+ * dP_ij = dout_i . v_j, D_i = dout_i . out_i and dlogit_ij = P_ij (dP_ij - D_i):
+ * dL/dl_j = sum g_h dlogit_ij, dL/dg_h = sum l_j dlogit_ij, dL/dtau_h =
+ * -sum dlogit_ij (q_i . k_j) / (sqrt(head_dim) tau_h^2).  Gradients with respect
+ * to q, k and v are not computed.
+ *   lse        [Hq, M] natural-log LSE from tg_gated_attention (required)
+ *   logsig     [M] (required: without the bias there is no gate gradient)
+ *   workspace  device scratch of tg_attention_backward_workspace_bytes bytes,
+ *              16-byte aligned (TG_ERR_WORKSPACE when smaller)
+ *   algo       tg_algo (TG_ALGO_TCGEN05 needs bf16)
+ * Other arguments, layouts and errors as tg_gated_attention.  Results are summed
+ * with floating-point atomics, so the last bits may differ between calls.
+ */
+TG_API tg_status tg_gated_attention_backward(const void* q, const void* k, const void* v,
+                                             tg_dtype dtype, int32_t batch,
+                                             const int32_t* cu_kept_h, int32_t n_q_heads,
+                                             int32_t n_kv_heads, int32_t head_dim,
+                                             const float* logsig, const float* gain,
+                                             const float* temp, const void* out, const float* lse,
+                                             const void* dout, float* d_logsig, float* d_z_kept,
+                                             float* d_gain, float* d_temp, void* workspace,
+                                             size_t workspace_bytes, int32_t algo,
+                                             tg_stream_t stream);
+
+/* Workspace bytes tg_gated_attention_backward needs for this batch (host-only). */
+TG_API tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,
+                                                       int32_t n_q_heads, size_t* bytes_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,8 @@ __all__ = [
     "TG_BF16", "TG_FP32", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "TokenGateError",
     "library", "kept_offsets", "gate_score", "topk_select", "compact_gather", "gated_attention",
     "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
-    "attention_kernel", "topk_select_multi", "random_select",
+    "attention_kernel", "topk_select_multi", "random_select", "gated_attention_backward",
+    "attention_backward_workspace_bytes",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -40,6 +41,7 @@ EXPORTED_SYMBOLS = (
     "tg_kept_offsets", "tg_gate_score", "tg_topk_select", "tg_compact_gather",
     "tg_gated_attention", "tg_attention_workspace_bytes", "tg_attention_kernel",
     "tg_gated_attention_noalloc", "tg_topk_select_multi", "tg_random_select",
+    "tg_gated_attention_backward", "tg_attention_backward_workspace_bytes",
 )
 MAX_BUDGETS = 8
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
@@ -96,6 +98,11 @@ def library():
                                       ctypes.POINTER(ctypes.c_int32)]
     L.tg_gated_attention_noalloc.argtypes = [_vp, _vp, _vp, ctypes.c_int, _i32, _i32p, _i32, _i32,
                                              _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+    L.tg_gated_attention_backward.argtypes = [_vp, _vp, _vp, ctypes.c_int, _i32, _i32p, _i32, _i32,
+                                              _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                              _vp, _vp, ctypes.c_size_t, _i32, _vp]
+    L.tg_attention_backward_workspace_bytes.argtypes = [_i32, _i32p, _i32,
+                                                        ctypes.POINTER(ctypes.c_size_t)]
     for name in EXPORTED_SYMBOLS:
         if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -326,6 +333,40 @@ def gated_attention(q, k, v, cu_kept_host, logsig=None, gain=None, temp=None, ou
         _ptr(gain), _ptr(temp), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, algo,
         _stream(q.device)))
     return out, lse
+
+
+def attention_backward_workspace_bytes(cu_kept_host, n_q_heads):
+    """Device scratch bytes gated_attention_backward needs for this batch."""
+    cu, cu_p = _host_i32(cu_kept_host)
+    out = ctypes.c_size_t(0)
+    _check("tg_attention_backward_workspace_bytes", library().tg_attention_backward_workspace_bytes(
+        len(cu) - 1, cu_p, n_q_heads, ctypes.byref(out)))
+    return int(out.value)
+
+
+def gated_attention_backward(q, k, v, cu_kept_host, logsig, gain, temp, out, lse, dout,
+                             algo=ALGO_AUTO, workspace=None):
+    """Gradient of a loss through gated_attention with respect to the log-gates
+    (and the kept rows' gate scores), the gains and the temperatures.
+
+    dout = dL/dout [M, Hq, d]; out, lse = the forward's outputs (lse [Hq, M]).
+    Returns (d_logsig [M], d_z_kept [M], d_gain [Hq], d_temp [Hq]), fp32 device.
+    """
+    _need_cuda(q, k, v, logsig, gain, temp, out, lse, dout)
+    M, Hq, dh = q.shape
+    Hkv = k.shape[1]
+    cu, cu_p = _host_i32(cu_kept_host)
+    if workspace is None:
+        workspace = torch.empty(attention_backward_workspace_bytes(cu, Hq), dtype=torch.uint8,
+                                device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    d_l, d_z = torch.empty(M, **f32), torch.empty(M, **f32)
+    d_g, d_t = torch.empty(Hq, **f32), torch.empty(Hq, **f32)
+    _check("tg_gated_attention_backward", library().tg_gated_attention_backward(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), len(cu) - 1, cu_p, Hq, Hkv, dh, _ptr(logsig),
+        _ptr(gain), _ptr(temp), _ptr(out), _ptr(lse), _ptr(dout), _ptr(d_l), _ptr(d_z), _ptr(d_g),
+        _ptr(d_t), _ptr(workspace), workspace.numel(), algo, _stream(q.device)))
+    return d_l, d_z, d_g, d_t
 
 
 def gated_prefill(h, q, k, v, W1, b1, w2, b2, gain, temp, cu_seqlens, doc_begin, doc_end,

@@ -418,4 +418,54 @@ tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dty
                         out, lse, workspace, workspace_bytes, st);
 }
 
+tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,
+                                                int32_t n_q_heads, size_t* bytes_out) {
+  if (!bytes_out) return set_error(TG_ERR_INVALID_ARG, "bytes_out is NULL");
+  PromptTable t;
+  int max_len = 0;
+  tg_status r = build_kept_table(batch, cu_kept_h, &t, &max_len);
+  if (r != TG_OK) return r;
+  if (n_q_heads <= 0) return set_error(TG_ERR_SHAPE, "n_q_heads=%d", n_q_heads);
+  *bytes_out = attn_bwd_workspace_bytes(t.kept_start[batch], n_q_heads);
+  return TG_OK;
+}
+
+tg_status tg_gated_attention_backward(const void* q, const void* k, const void* v, tg_dtype dtype,
+                                      int32_t batch, const int32_t* cu_kept_h, int32_t n_q_heads,
+                                      int32_t n_kv_heads, int32_t head_dim, const float* logsig,
+                                      const float* gain, const float* temp, const void* out,
+                                      const float* lse, const void* dout, float* d_logsig,
+                                      float* d_z_kept, float* d_gain, float* d_temp,
+                                      void* workspace, size_t workspace_bytes, int32_t algo,
+                                      tg_stream_t stream) {
+  if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
+  PromptTable t;
+  int max_len = 0;
+  tg_status r = build_kept_table(batch, cu_kept_h, &t, &max_len);
+  if (r != TG_OK) return r;
+  if (n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0)
+    return set_error(TG_ERR_SHAPE, "n_q_heads=%d n_kv_heads=%d", n_q_heads, n_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(TG_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", head_dim);
+  if (algo < TG_ALGO_AUTO || algo > TG_ALGO_TCGEN05)
+    return set_error(TG_ERR_INVALID_ARG, "algo %d", algo);
+  const int64_t M = t.kept_start[batch];
+  if (M == 0) return TG_OK;
+  if (!q || !k || !v || !logsig || !gain || !temp || !out || !lse || !dout || !d_logsig ||
+      !d_z_kept || !d_gain || !d_temp || !workspace)
+    return set_error(TG_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(workspace))
+    return set_error(TG_ERR_ALIGNMENT, "q/k/v/out/dout/workspace must be 16-byte aligned");
+  const size_t need = attn_bwd_workspace_bytes(M, n_q_heads);
+  if (workspace_bytes < need)
+    return set_error(TG_ERR_WORKSPACE, "attention backward workspace: %zu bytes given, %zu needed",
+                     workspace_bytes, need);
+  if (algo == TG_ALGO_TCGEN05 && dtype != TG_BF16)
+    return set_error(TG_ERR_UNSUPPORTED, "tcgen05 attention backward needs bf16");
+  return launch_attn_bwd(q, k, v, out, dout, dtype, t, n_q_heads, n_kv_heads, head_dim, logsig,
+                         gain, temp, lse, d_logsig, d_z_kept, d_gain, d_temp, workspace,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

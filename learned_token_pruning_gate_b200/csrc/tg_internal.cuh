@@ -60,6 +60,14 @@ tg_status launch_attn_tc(const void* q, const void* k, const void* v, const Prom
                          int max_len, int hq, int hkv, int dh, const float* logsig,
                          const float* gain, const float* temp, void* out, float* lse,
                          void* workspace, size_t workspace_bytes, cudaStream_t st);
+// Backward of the gated attention (log-gates, gains, temperatures); workspace of
+// attn_bwd_workspace_bytes (D per row and head, per-head accumulators).
+tg_status launch_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                          const void* dout, tg_dtype dt, const PromptTable& pt, int hq, int hkv,
+                          int dh, const float* logsig, const float* gain, const float* temp,
+                          const float* lse, float* d_logsig, float* d_z_kept, float* d_gain,
+                          float* d_temp, void* workspace, cudaStream_t st);
+size_t attn_bwd_workspace_bytes(int64_t m_total, int hq);
 // Workspace the tensor-core attention uses to split long items on this device (0 = none).
 size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh);
 // The tg_attn_kernel the tensor-core attention launches for this batch.

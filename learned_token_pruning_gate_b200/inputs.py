@@ -187,6 +187,12 @@ def random_scores(n: int, seed: int, ties: bool = True, specials: bool = True) -
     return z
 
 
+def attention_output_grad(M, Hq, dh, seed, dtype="bf16"):
+    """A seeded upstream gradient dL/dout [M, Hq, dh] for the attention backward."""
+    rng = np.random.Generator(np.random.Philox(seed + 7919))
+    return torch.from_numpy(_normal(rng, (M, Hq, dh))).to(_tdtype(dtype))
+
+
 def attention_inputs(M_list, Hq, Hkv, dh, seed, dtype="bf16", bias=True):
     """Compacted-layout attention inputs drawn directly (for stage-level tests)."""
     rng = np.random.Generator(np.random.Philox(seed))

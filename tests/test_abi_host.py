@@ -245,3 +245,38 @@ def test_budget_sweep_and_random_select_validation(L):
     big, big_p = _arr([0, 400000])
     s0, s0_p = _arr([0])
     assert r(FAKE, 1, big_p, s0_p, s0_p, k1_p, FAKE, FAKE, None) == UNSUP     # too long
+
+
+def test_attention_backward_validation(L):
+    """The backward rejects bad arguments before launching anything."""
+    _, ck = _arr([0, 300])
+    need = ctypes.c_size_t(0)
+    assert L.tg_attention_backward_workspace_bytes(1, ck, 16, ctypes.byref(need)) == OK
+    # D for 300 rows x 16 heads plus the per-head accumulators, 256-byte rounded
+    assert need.value >= 300 * 16 * 4 + 2 * 16 * 4 and need.value % 256 == 0
+    assert L.tg_attention_backward_workspace_bytes(1, ck, 0, ctypes.byref(need)) == SHAPE
+    assert L.tg_attention_backward_workspace_bytes(1, ck, 16, None) == INVALID
+    L.tg_attention_backward_workspace_bytes(1, ck, 16, ctypes.byref(need))
+    b = L.tg_gated_attention_backward
+
+    def call(dtype=0, hq=16, hkv=8, dh=128, logsig=FAKE, lse=FAKE, ws=FAKE, ws_bytes=None,
+             algo=0, q=FAKE):
+        return b(q, FAKE, FAKE, dtype, 1, ck, hq, hkv, dh, logsig, FAKE, FAKE, FAKE, lse, FAKE,
+                 FAKE, FAKE, FAKE, FAKE, ws, need.value if ws_bytes is None else ws_bytes, algo,
+                 None)
+
+    assert call(dtype=7) == DTYPE
+    assert call(hkv=6) == SHAPE
+    assert call(dh=96) == UNSUP
+    assert call(algo=9) == INVALID
+    assert call(logsig=None) == INVALID  # no bias, no gate gradient
+    assert call(lse=None) == INVALID
+    assert call(ws=None) == INVALID
+    assert call(q=FAKE_ODD) == ALIGN
+    assert call(ws_bytes=need.value - 16) == WORKSPACE
+    assert b"needed" in L.tg_last_error_message()
+    assert call(dtype=1, algo=2) == UNSUP  # tcgen05 needs bf16
+    # nothing kept: nothing to do, nothing launched
+    _, ck0 = _arr([0, 0])
+    assert b(None, None, None, 0, 1, ck0, 16, 8, 128, None, None, None, None, None, None, None,
+             None, None, None, None, 0, 0, None) == OK
