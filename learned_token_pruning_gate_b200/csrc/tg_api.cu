@@ -464,7 +464,7 @@ tg_status tg_gated_attention_backward(const void* q, const void* k, const void* 
   if (algo == TG_ALGO_TCGEN05 && dtype != TG_BF16)
     return set_error(TG_ERR_UNSUPPORTED, "tcgen05 attention backward needs bf16");
   return launch_attn_bwd(q, k, v, out, dout, dtype, t, n_q_heads, n_kv_heads, head_dim, logsig,
-                         gain, temp, lse, d_logsig, d_z_kept, d_gain, d_temp, workspace,
+                         gain, temp, lse, d_logsig, d_z_kept, d_gain, d_temp, workspace, algo,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -66,7 +66,7 @@ tg_status launch_attn_bwd(const void* q, const void* k, const void* v, const voi
                           const void* dout, tg_dtype dt, const PromptTable& pt, int hq, int hkv,
                           int dh, const float* logsig, const float* gain, const float* temp,
                           const float* lse, float* d_logsig, float* d_z_kept, float* d_gain,
-                          float* d_temp, void* workspace, cudaStream_t st);
+                          float* d_temp, void* workspace, int algo, cudaStream_t st);
 size_t attn_bwd_workspace_bytes(int64_t m_total, int hq);
 // Workspace the tensor-core attention uses to split long items on this device (0 = none).
 size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh);
