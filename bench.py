@@ -414,8 +414,18 @@ def run_ncu_case(args):
     layer = GatedLayer(d(inp.h), d(inp.q), d(inp.k), d(inp.v), d(inp.W1), d(inp.b1), d(inp.w2),
                        inp.b2, d(inp.gain), d(inp.temp), inp.cu_seqlens, inp.doc_begin,
                        inp.doc_end, inp.budget, rope_theta=w.rope_theta)
+    bwd = None
+    if args.backward:
+        o, lse = tg.gated_attention(layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host, layer.logsig,
+                                    layer.gain, layer.temp, want_lse=True)
+        dout = gen.attention_output_grad(layer.M, w.n_q_heads, w.head_dim, w.seed, w.dtype).cuda()
+        bwd = lambda: tg.gated_attention_backward(  # noqa: E731
+            layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host, layer.logsig, layer.gain,
+            layer.temp, o, lse, dout)
     for _ in range(args.steps):
         layer.run()
+        if bwd:
+            bwd()
     torch.cuda.synchronize()
     if tg.device_status() != 0:
         raise SystemExit("a kernel reported a timed-out wait")
@@ -488,7 +498,20 @@ def run_extras(args):
     no_bias = timed(lambda: tg.gated_attention(layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host,
                                                None, layer.gain, layer.temp, out=layer.out,
                                                workspace=ws), 20)
-    del layer
+    # backward of the gated attention w.r.t. log-gates, gains, temperatures (training the
+    # gate): S and dP over the causal triangle, the same flop count as the forward
+    Mk = sum(w.kept_lengths())
+    o_f, lse_f = tg.gated_attention(layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host,
+                                    layer.logsig, layer.gain, layer.temp, want_lse=True,
+                                    workspace=ws)
+    dout = gen.attention_output_grad(Mk, w.n_q_heads, w.head_dim, w.seed, w.dtype).to(dev)
+    bws = torch.empty(tg.attention_backward_workspace_bytes(layer.cu_kept_host, w.n_q_heads),
+                      dtype=torch.uint8, device=dev)
+    bwd_us = timed(lambda: tg.gated_attention_backward(
+        layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host, layer.logsig, layer.gain, layer.temp,
+        o_f, lse_f, dout, workspace=bws), 20)
+    kept_flops = float(sum(2.0 * w.head_dim * w.n_q_heads * m * (m + 1) for m in w.kept_lengths()))
+    del layer, o_f, lse_f, dout, bws
     torch.cuda.synchronize()
     # ungated: every token of every prompt attends causally, no bias (the layer without a gate)
     q, k, v = res[1], res[2], res[3]
@@ -517,6 +540,10 @@ def run_extras(args):
         "ungated_attention": {"us": round(ungated, 2), "tflops": round(full_flops / ungated / 1e6, 1),
                               "frac_measured_bf16": round(full_flops / ungated / 1e6 / _peaks()["bf16"], 4)},
         "speedup_vs_ungated_attention": round(ungated / gated_total, 2),
+        "attention_backward": {"us": round(bwd_us, 2),
+                               "tflops": round(kept_flops / bwd_us / 1e6, 1),
+                               "frac_measured_bf16": round(kept_flops / bwd_us / 1e6 / _peaks()["bf16"], 4),
+                               "grads": "log-gates (and kept scores), gains, temperatures"},
         "selection": {"budget_sweep_8_one_launch_us": round(sweep_one, 2),
                       "budget_sweep_8_separate_launches_us": round(sweep_sep, 2),
                       "random_k_us": round(rand_us, 2), "topk_us": round(stage_us["topk"], 2)},
@@ -548,6 +575,8 @@ def main():
                     help="print bias overhead, ungated full-N attention and memory figures")
     ap.add_argument("--ncu-case", action="store_true",
                     help="untimed: run --steps plain steps of the workload (profiling)")
+    ap.add_argument("--backward", action="store_true",
+                    help="with --ncu-case: also run the attention backward after each step")
     args = ap.parse_args()
     if args.ncu_case:
         run_ncu_case(args)
