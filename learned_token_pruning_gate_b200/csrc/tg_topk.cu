@@ -11,7 +11,10 @@
 //     order-preserving 32-bit keys (padded by one word per 32 so both strided
 //     and per-thread-contiguous walks are free of bank conflicts) and builds the
 //     first radix histogram while loading.
-//  2. Three radix passes (11, 11, 10 bits) find the K-th largest key T.  Every
+//  2. Up to three radix passes (11, 11, 10 bits) find the K-th largest key T;
+//     when every key of a pass's boundary bin is kept, the low bits cannot
+//     change the set and the search stops there (T then fixes only the high
+//     bits; usually the last pass is skipped for continuous scores).  Every
 //     cross-CTA step is a one-way write: each CTA adds its non-zero bins into
 //     the leader CTA's histogram with remote shared-memory atomics, a cluster
 //     barrier publishes them, the leader scans and pushes the chosen digit into
@@ -96,7 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
   __shared__ uint32_t s_hist[kBins];           // this CTA's histogram of the current pass
   __shared__ uint32_t s_total[2][kBins];       // cluster totals (used in the leader only)
   __shared__ uint32_t s_scan[33];
-  __shared__ uint32_t s_sel[2];                // digit, count above (pushed by the leader)
+  __shared__ uint32_t s_sel[3];                // digit, count above, count in the digit's bin
   __shared__ uint32_t s_cnt[kMaxCluster][2];   // lower-ranked CTAs' (sure, tie) counts
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -136,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
   cluster.sync();  // every CTA has started and zeroed its totals
 
   uint32_t T = 0, need = 0;
+  uint32_t hmask = 0xFFFFFFFFu;  // key bits the threshold T fixes
   if (mode == 2) {
     uint32_t* lead_sel = cluster.map_shared_rank(s_sel, 0);
     uint32_t prefix = 0, k_rem = static_cast<uint32_t>(kk);
@@ -185,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
                 uint32_t* sel = cluster.map_shared_rank(s_sel, rr);
                 sel[0] = digit;
                 sel[1] = above;
+                sel[2] = cnt[j];
               }
               break;
             }
@@ -195,10 +200,16 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
       cluster.sync();  // the chosen digit is visible everywhere
       prefix |= s_sel[0] << shift;
       k_rem -= s_sel[1];
+      if (s_sel[2] == k_rem) {
+        // every key of the boundary bin is kept: the remaining low bits cannot
+        // change the set, so stop here (the same decision in every CTA)
+        hmask = 0xFFFFFFFFu << shift;
+        break;
+      }
     }
     (void)lead_sel;
     T = prefix;
-    need = k_rem;  // how many keys == T to keep, lowest indices first
+    need = k_rem;  // how many keys whose fixed bits equal T to keep, lowest indices first
   }
 
   // ---- ordered compaction -------------------------------------------------
@@ -210,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
     const int32_t pos = lo + i;
     const bool doc = pos >= ds && pos < de;
     const uint32_t key = s_keys[padded(i)];
-    gt += (!doc || mode == 1 || (mode == 2 && key > T)) ? 1u : 0u;
-    eq += (doc && mode == 2 && key == T) ? 1u : 0u;
+    gt += (!doc || mode == 1 || (mode == 2 && (key & hmask) > T)) ? 1u : 0u;
+    eq += (doc && mode == 2 && (key & hmask) == T) ? 1u : 0u;
   }
   // packed (ties << 16 | sure) fits: at most 45056 keys per CTA
   uint32_t tot = 0;
@@ -237,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
     const int32_t pos = lo + i;
     const bool doc = pos >= ds && pos < de;
     const uint32_t key = s_keys[padded(i)];
-    bool keep = !doc || mode == 1 || (mode == 2 && key > T);
-    if (doc && mode == 2 && key == T) {
+    bool keep = !doc || mode == 1 || (mode == 2 && (key & hmask) > T);
+    if (doc && mode == 2 && (key & hmask) == T) {
       keep = tie_rank < need_here;
       ++tie_rank;
     }
