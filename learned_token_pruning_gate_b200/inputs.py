@@ -187,6 +187,33 @@ def random_scores(n: int, seed: int, ties: bool = True, specials: bool = True) -
     return z
 
 
+def stack_inputs(M_list, n_layers, d_model, Hq, Hkv, dh, inter, seed, dtype="bf16", pos_span=4):
+    """A compacted residual, the kept rows' original positions, log-gates and the
+    random-init weights of n_layers Qwen3-shaped upper layers (stage-level tests
+    and the stack benchmark).  Positions: sorted distinct draws from
+    [0, pos_span * M_b) per prompt (a kept set of about 1 row in pos_span)."""
+    rng = np.random.Generator(np.random.Philox(seed + 104729))
+    dt = _tdtype(dtype)
+    M = int(sum(M_list))
+    cu = np.zeros(len(M_list) + 1, np.int32)
+    cu[1:] = np.cumsum(M_list)
+    pos = np.concatenate([np.sort(rng.choice(max(pos_span * m, 1), size=m, replace=False))
+                          for m in M_list]).astype(np.int32) if M else np.zeros(0, np.int32)
+    x0 = torch.from_numpy(_normal(rng, (M, d_model))).to(dt)
+    ls = torch.from_numpy(-np.abs(_normal(rng, (M,), 2.0)))
+    w = lambda *shape: torch.from_numpy(_normal(rng, shape, 0.02)).to(dt)  # noqa: E731
+    norm_w = lambda n: torch.from_numpy((1.0 + _normal(rng, (n,), 0.1)).astype(np.float32)).to(dt)  # noqa: E731
+    layers = []
+    for _ in range(n_layers):
+        layers.append(dict(
+            w_ln1=norm_w(d_model), wqkv=w((Hq + 2 * Hkv) * dh, d_model), w_qn=norm_w(dh),
+            w_kn=norm_w(dh), wo=w(d_model, Hq * dh), w_ln2=norm_w(d_model), wg=w(inter, d_model),
+            wu=w(inter, d_model), wd=w(d_model, inter),
+            gain=torch.from_numpy(rng.uniform(0.0, 1.0, Hq).astype(np.float32)),
+            temp=torch.from_numpy(rng.uniform(0.8, 1.2, Hq).astype(np.float32))))
+    return cu, pos, x0, ls, layers
+
+
 def attention_output_grad(M, Hq, dh, seed, dtype="bf16"):
     """A seeded upstream gradient dL/dout [M, Hq, dh] for the attention backward."""
     rng = np.random.Generator(np.random.Philox(seed + 7919))
