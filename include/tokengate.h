@@ -327,6 +327,49 @@ TG_API tg_status tg_gated_attention_backward(const void* q, const void* k, const
                                              size_t workspace_bytes, int32_t algo,
                                              tg_stream_t stream);
 
+/*
+ * Steps of a stack of gated upper layers.  Every attention layer above the gate
+ * keeps working on the same kept rows and creates KV only for them (TokenGate,
+ * "How it works"), each with its own gain and temperature on the shared
+ * log-gates.  The layers are Qwen3-shaped: RMSNorm, a fused QKV projection,
+ * per-head RMSNorm of q and k, RoPE at the kept rows' original positions,
+ * tg_gated_attention, an output projection, RMSNorm and a SwiGLU MLP.  The
+ * projections are plain GEMMs left to the caller (cuBLAS); these calls do the
+ * rest.  Row-major, contiguous, device pointers; dtype TG_BF16 or TG_FP32 with
+ * fp32 arithmetic.
+ *
+ * tg_rmsnorm: out[r, c] = x[r, c] / sqrt(mean_c x[r, c]^2 + eps) * weight[c].
+ *   x, out [rows, dim] (out may equal x), weight [dim].
+ */
+TG_API tg_status tg_rmsnorm(const void* x, const void* weight, void* out, tg_dtype dtype,
+                            int64_t rows, int32_t dim, float eps, tg_stream_t stream);
+
+/*
+ * tg_qkv_rope_emit: split of a fused QKV projection of the kept rows.
+ *   qkv      [M, (n_q_heads + 2 n_kv_heads) * head_dim]: q heads, then k heads, then v
+ *   q_out    [M, n_q_heads, head_dim]    RMSNorm(q_h) * q_norm_w, then RoPE
+ *   k_out    [M, n_kv_heads, head_dim]   RMSNorm(k_h) * k_norm_w, then RoPE (the KV cache
+ *                                        slot of this layer, compacted)
+ *   v_out    [M, n_kv_heads, head_dim]   v as it is (the cache slot)
+ *   RoPE: rotate-half pairs (i, i + head_dim/2), angle pos * rope_theta^(-2i/head_dim)
+ *   with pos = kept_idx[i] - cu_seqlens_h[b] the row's original position in its
+ *   prompt b (cu_kept_h gives the kept rows of each prompt, host arrays as in
+ *   tg_compact_gather).  head_dim 64 or 128.
+ */
+TG_API tg_status tg_qkv_rope_emit(const void* qkv, tg_dtype dtype, int32_t batch,
+                                  const int32_t* cu_seqlens_h, const int32_t* cu_kept_h,
+                                  const int32_t* kept_idx, int32_t n_q_heads, int32_t n_kv_heads,
+                                  int32_t head_dim, const void* q_norm_w, const void* k_norm_w,
+                                  float eps, double rope_theta, void* q_out, void* k_out,
+                                  void* v_out, tg_stream_t stream);
+
+/*
+ * tg_swiglu: out[r, c] = SiLU(gate_up[r, c]) * gate_up[r, inter + c], SiLU(g) = g / (1 + e^-g).
+ *   gate_up [rows, 2 inter] (the fused gate and up projections), out [rows, inter].
+ */
+TG_API tg_status tg_swiglu(const void* gate_up, void* out, tg_dtype dtype, int64_t rows,
+                           int32_t inter, tg_stream_t stream);
+
 /* Workspace bytes tg_gated_attention_backward needs for this batch (host-only). */
 TG_API tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,
                                                        int32_t n_q_heads, size_t* bytes_out);

@@ -25,7 +25,7 @@ __all__ = [
     "library", "kept_offsets", "gate_score", "topk_select", "compact_gather", "gated_attention",
     "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
     "attention_kernel", "topk_select_multi", "random_select", "gated_attention_backward",
-    "attention_backward_workspace_bytes",
+    "attention_backward_workspace_bytes", "rmsnorm", "qkv_rope_emit", "swiglu",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -41,7 +41,8 @@ EXPORTED_SYMBOLS = (
     "tg_kept_offsets", "tg_gate_score", "tg_topk_select", "tg_compact_gather",
     "tg_gated_attention", "tg_attention_workspace_bytes", "tg_attention_kernel",
     "tg_gated_attention_noalloc", "tg_topk_select_multi", "tg_random_select",
-    "tg_gated_attention_backward", "tg_attention_backward_workspace_bytes",
+    "tg_gated_attention_backward", "tg_attention_backward_workspace_bytes", "tg_rmsnorm",
+    "tg_qkv_rope_emit", "tg_swiglu",
 )
 MAX_BUDGETS = 8
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
@@ -103,6 +104,10 @@ def library():
                                               _vp, _vp, ctypes.c_size_t, _i32, _vp]
     L.tg_attention_backward_workspace_bytes.argtypes = [_i32, _i32p, _i32,
                                                         ctypes.POINTER(ctypes.c_size_t)]
+    L.tg_rmsnorm.argtypes = [_vp, _vp, _vp, ctypes.c_int, _i64, _i32, _f32, _vp]
+    L.tg_qkv_rope_emit.argtypes = [_vp, ctypes.c_int, _i32, _i32p, _i32p, _vp, _i32, _i32, _i32,
+                                   _vp, _vp, _f32, ctypes.c_double, _vp, _vp, _vp, _vp]
+    L.tg_swiglu.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i32, _vp]
     for name in EXPORTED_SYMBOLS:
         if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -367,6 +372,48 @@ def gated_attention_backward(q, k, v, cu_kept_host, logsig, gain, temp, out, lse
         _ptr(gain), _ptr(temp), _ptr(out), _ptr(lse), _ptr(dout), _ptr(d_l), _ptr(d_z), _ptr(d_g),
         _ptr(d_t), _ptr(workspace), workspace.numel(), algo, _stream(q.device)))
     return d_l, d_z, d_g, d_t
+
+
+def rmsnorm(x, weight, eps=1e-6, out=None):
+    """x / sqrt(mean(x^2) + eps) * weight over the last axis of x [rows, dim]."""
+    _need_cuda(x, weight)
+    rows, dim = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check("tg_rmsnorm", library().tg_rmsnorm(_ptr(x), _ptr(weight), _ptr(out), _dtype_code(x),
+                                              rows, dim, eps, _stream(x.device)))
+    return out
+
+
+def qkv_rope_emit(qkv, cu_seqlens, cu_kept_host, kept_idx, n_q_heads, n_kv_heads, head_dim,
+                  q_norm_w, k_norm_w, eps=1e-6, rope_theta=1e6, q_out=None, k_out=None,
+                  v_out=None):
+    """Split a fused QKV projection [M, (Hq + 2 Hkv) d] into q (per-head RMSNorm,
+    RoPE), k (same; the layer's KV-cache slot) and v.  Returns (q, k, v)."""
+    _need_cuda(qkv, kept_idx, q_norm_w, k_norm_w)
+    M = qkv.shape[0]
+    cu, cu_p = _host_i32(cu_seqlens)
+    ck, ck_p = _host_i32(cu_kept_host)
+    mk = lambda h: torch.empty((M, h, head_dim), dtype=qkv.dtype, device=qkv.device)  # noqa: E731
+    q_out = mk(n_q_heads) if q_out is None else q_out
+    k_out = mk(n_kv_heads) if k_out is None else k_out
+    v_out = mk(n_kv_heads) if v_out is None else v_out
+    _check("tg_qkv_rope_emit", library().tg_qkv_rope_emit(
+        _ptr(qkv), _dtype_code(qkv), len(cu) - 1, cu_p, ck_p, _ptr(kept_idx), n_q_heads, n_kv_heads,
+        head_dim, _ptr(q_norm_w), _ptr(k_norm_w), eps, float(rope_theta), _ptr(q_out), _ptr(k_out),
+        _ptr(v_out), _stream(qkv.device)))
+    return q_out, k_out, v_out
+
+
+def swiglu(gate_up, out=None):
+    """SiLU(gate) * up of a fused [rows, 2 inter] projection."""
+    _need_cuda(gate_up)
+    rows, two = gate_up.shape
+    if out is None:
+        out = torch.empty((rows, two // 2), dtype=gate_up.dtype, device=gate_up.device)
+    _check("tg_swiglu", library().tg_swiglu(_ptr(gate_up), _ptr(out), _dtype_code(gate_up), rows,
+                                            two // 2, _stream(gate_up.device)))
+    return out
 
 
 def gated_prefill(h, q, k, v, W1, b1, w2, b2, gain, temp, cu_seqlens, doc_begin, doc_end,

@@ -418,6 +418,59 @@ tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dty
                         out, lse, workspace, workspace_bytes, st);
 }
 
+tg_status tg_rmsnorm(const void* x, const void* weight, void* out, tg_dtype dtype, int64_t rows,
+                     int32_t dim, float eps, tg_stream_t stream) {
+  if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
+  if (rows < 0 || dim <= 0) return set_error(TG_ERR_SHAPE, "rows=%lld dim=%d", static_cast<long long>(rows), dim);
+  if (!(eps >= 0.0f)) return set_error(TG_ERR_INVALID_ARG, "eps must be >= 0");
+  if (rows == 0) return TG_OK;
+  if (!x || !weight || !out) return set_error(TG_ERR_INVALID_ARG, "null pointer");
+  return launch_rmsnorm(x, weight, out, dtype, rows, dim, eps, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tg_status tg_qkv_rope_emit(const void* qkv, tg_dtype dtype, int32_t batch, const int32_t* cu_seqlens_h,
+                           const int32_t* cu_kept_h, const int32_t* kept_idx, int32_t n_q_heads,
+                           int32_t n_kv_heads, int32_t head_dim, const void* q_norm_w,
+                           const void* k_norm_w, float eps, double rope_theta, void* q_out,
+                           void* k_out, void* v_out, tg_stream_t stream) {
+  if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
+  PromptTable t;
+  int max_len = 0;
+  tg_status r = build_kept_table(batch, cu_kept_h, &t, &max_len);
+  if (r != TG_OK) return r;
+  if (!cu_seqlens_h) return set_error(TG_ERR_INVALID_ARG, "cu_seqlens_h is null");
+  if (cu_seqlens_h[0] != 0) return set_error(TG_ERR_INVALID_ARG, "cu_seqlens[0] must be 0");
+  for (int b = 0; b < batch; ++b) {
+    const int64_t n = static_cast<int64_t>(cu_seqlens_h[b + 1]) - cu_seqlens_h[b];
+    if (n < 0) return set_error(TG_ERR_INVALID_ARG, "cu_seqlens decreases at prompt %d", b);
+    if (t.kept_start[b + 1] - t.kept_start[b] > n)
+      return set_error(TG_ERR_INVALID_ARG, "prompt %d keeps more rows than it has", b);
+    t.start[b] = cu_seqlens_h[b];
+  }
+  t.start[batch] = cu_seqlens_h[batch];
+  if (n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0)
+    return set_error(TG_ERR_SHAPE, "n_q_heads=%d n_kv_heads=%d", n_q_heads, n_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(TG_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", head_dim);
+  if (!(rope_theta > 1.0) || !(eps >= 0.0f)) return set_error(TG_ERR_INVALID_ARG, "rope_theta / eps");
+  if (t.kept_start[batch] == 0) return TG_OK;
+  if (!qkv || !kept_idx || !q_norm_w || !k_norm_w || !q_out || !k_out || !v_out)
+    return set_error(TG_ERR_INVALID_ARG, "null pointer");
+  return launch_qkv_emit(qkv, dtype, t, kept_idx, n_q_heads, n_kv_heads, head_dim, q_norm_w,
+                         k_norm_w, eps, rope_theta, q_out, k_out, v_out,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+tg_status tg_swiglu(const void* gate_up, void* out, tg_dtype dtype, int64_t rows, int32_t inter,
+                    tg_stream_t stream) {
+  if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
+  if (rows < 0 || inter <= 0)
+    return set_error(TG_ERR_SHAPE, "rows=%lld inter=%d", static_cast<long long>(rows), inter);
+  if (rows == 0) return TG_OK;
+  if (!gate_up || !out) return set_error(TG_ERR_INVALID_ARG, "null pointer");
+  return launch_swiglu(gate_up, out, dtype, rows, inter, reinterpret_cast<cudaStream_t>(stream));
+}
+
 tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,
                                                 int32_t n_q_heads, size_t* bytes_out) {
   if (!bytes_out) return set_error(TG_ERR_INVALID_ARG, "bytes_out is NULL");

@@ -68,6 +68,14 @@ tg_status launch_attn_bwd(const void* q, const void* k, const void* v, const voi
                           const float* lse, float* d_logsig, float* d_z_kept, float* d_gain,
                           float* d_temp, void* workspace, int algo, cudaStream_t st);
 size_t attn_bwd_workspace_bytes(int64_t m_total, int hq);
+// Element-wise steps of the gated upper-layer stack.
+tg_status launch_rmsnorm(const void* x, const void* w, void* y, tg_dtype dt, int64_t rows, int dim,
+                         float eps, cudaStream_t st);
+tg_status launch_qkv_emit(const void* qkv, tg_dtype dt, const PromptTable& pt, const int32_t* kept_idx,
+                          int hq, int hkv, int dh, const void* w_qn, const void* w_kn, float eps,
+                          double theta, void* q_out, void* k_out, void* v_out, cudaStream_t st);
+tg_status launch_swiglu(const void* gu, void* h, tg_dtype dt, int64_t rows, int inter,
+                        cudaStream_t st);
 // Workspace the tensor-core attention uses to split long items on this device (0 = none).
 size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh);
 // The tg_attn_kernel the tensor-core attention launches for this batch.

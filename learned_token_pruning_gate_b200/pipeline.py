@@ -14,7 +14,8 @@ import numpy as np
 import torch
 
 from . import (ALGO_AUTO, GatherTensor, _check, _dtype_code, _host_i32,
-               attention_workspace_bytes, kept_offsets, library)
+               attention_workspace_bytes, gated_attention, kept_offsets, library, qkv_rope_emit,
+               rmsnorm, swiglu)
 
 
 class GatedLayer:
@@ -133,3 +134,52 @@ class GatedLayer:
             attn_bytes=float(self.M * row_bytes - self.M * self.d * esz
                              + self.M * self.Hq * self.dh * esz + 4 * self.M),
         )
+
+
+class GatedStack:
+    """Upper layers above the gate over the kept rows: every layer reuses the kept
+    set and the log-gates, with its own gain and temperature, and emits its k and
+    v (post-RoPE) into a compacted KV cache [layers, M, Hkv, d].  Qwen3-shaped
+    layers (RMSNorm, fused QKV, per-head q/k RMSNorm, RoPE at the original
+    positions, gated attention, output projection, RMSNorm, SwiGLU MLP); the
+    projections are cuBLAS GEMMs (torch.mm), every other step a libtokengate call.
+
+    layers: list of dicts of device tensors w_ln1, wqkv, w_qn, w_kn, wo, w_ln2, wg,
+    wu, wd (dtype of the activations), gain, temp (fp32).
+    """
+
+    def __init__(self, layers, n_q_heads, n_kv_heads, head_dim, cu_seqlens, cu_kept_host, kept_idx,
+                 logsig, rope_theta=1e6, eps=1e-6):
+        self.layers = layers
+        self.Hq, self.Hkv, self.dh = n_q_heads, n_kv_heads, head_dim
+        self.cu = np.asarray(cu_seqlens, np.int32)
+        self.ck = np.asarray(cu_kept_host, np.int32)
+        self.kept_idx, self.logsig = kept_idx, logsig
+        self.theta, self.eps = rope_theta, eps
+        self.M = int(self.ck[-1])
+        # fused [gate; up] weight per layer: one GEMM for both
+        self.wgu = [torch.cat([ly["wg"], ly["wu"]], 0) for ly in layers]
+        dev, dt = layers[0]["wqkv"].device, layers[0]["wqkv"].dtype
+        L, M = len(layers), self.M
+        self.cache_k = torch.empty((L, M, n_kv_heads, head_dim), dtype=dt, device=dev)
+        self.cache_v = torch.empty((L, M, n_kv_heads, head_dim), dtype=dt, device=dev)
+        self.q = torch.empty((M, n_q_heads, head_dim), dtype=dt, device=dev)
+        self.o = torch.empty((M, n_q_heads, head_dim), dtype=dt, device=dev)
+        nbytes = attention_workspace_bytes(self.ck, n_q_heads, n_kv_heads, head_dim, dt)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+
+    def run(self, x):
+        """x [M, d_model] (overwritten with the stack's output); returns (x, cache_k, cache_v)."""
+        M, Hq = self.M, self.Hq
+        for i, ly in enumerate(self.layers):
+            a = rmsnorm(x, ly["w_ln1"], self.eps)
+            qkv = torch.mm(a, ly["wqkv"].t())
+            qkv_rope_emit(qkv, self.cu, self.ck, self.kept_idx, Hq, self.Hkv, self.dh, ly["w_qn"],
+                             ly["w_kn"], self.eps, self.theta, q_out=self.q,
+                             k_out=self.cache_k[i], v_out=self.cache_v[i])
+            gated_attention(self.q, self.cache_k[i], self.cache_v[i], self.ck, self.logsig,
+                               ly["gain"], ly["temp"], out=self.o, workspace=self.ws)
+            x.addmm_(self.o.view(M, Hq * self.dh), ly["wo"].t())
+            b = rmsnorm(x, ly["w_ln2"], self.eps)
+            x.addmm_(swiglu(torch.mm(b, self.wgu[i].t())), ly["wd"].t())
+        return x, self.cache_k, self.cache_v
