@@ -511,6 +511,31 @@ def run_extras(args):
         layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host, layer.logsig, layer.gain, layer.temp,
         o_f, lse_f, dout, workspace=bws), 20)
     kept_flops = float(sum(2.0 * w.head_dim * w.n_q_heads * m * (m + 1) for m in w.kept_lengths()))
+    # a stack of 4 Qwen3-1.7B-shaped upper layers over the kept rows (random init):
+    # shared kept set and log-gates, per-layer gain and temperature, compacted KV cache
+    stack = None
+    if w.dtype == "bf16":
+        from learned_token_pruning_gate_b200.pipeline import GatedStack
+        n_up = 4
+        _, _, _, _, sl = gen.stack_inputs([1] * len(w.kept_lengths()), n_up, w.d_model, w.n_q_heads,
+                                          w.n_kv_heads, w.head_dim, 6144, w.seed, w.dtype)
+        sl = [{k_: v_.to(dev) for k_, v_ in ly.items()} for ly in sl]
+        st_ = GatedStack(sl, w.n_q_heads, w.n_kv_heads, w.head_dim, inp.cu_seqlens,
+                         layer.cu_kept_host, layer.kept_idx, layer.logsig, rope_theta=w.rope_theta)
+        xs = layer.h_c.clone()
+        stack_us = timed(lambda: st_.run(xs), 10)
+        # the same layers' attention alone (per layer, shared q/k/v buffers)
+        att_us = timed(lambda: [tg.gated_attention(st_.q, st_.cache_k[i], st_.cache_v[i],
+                                                   layer.cu_kept_host, layer.logsig, ly["gain"],
+                                                   ly["temp"], out=st_.o, workspace=st_.ws)
+                                for i, ly in enumerate(sl)], 10)
+        kv_c = int(st_.cache_k.numel() + st_.cache_v.numel()) * 2
+        stack = {"layers": n_up, "us": round(stack_us, 2), "us_per_layer": round(stack_us / n_up, 2),
+                 "attention_us": round(att_us, 2),
+                 "kv_cache_bytes": kv_c, "kv_cache_full_n_bytes": int(kv_c * w.total_tokens / Mk),
+                 "note": "Qwen3-1.7B-shaped (d 2048, 16/8 x 128, MLP 6144), random init; GEMMs "
+                         "cuBLAS, other steps libtokengate"}
+        del st_, xs, sl
     del layer, o_f, lse_f, dout, bws
     torch.cuda.synchronize()
     # ungated: every token of every prompt attends causally, no bias (the layer without a gate)
@@ -540,6 +565,7 @@ def run_extras(args):
         "ungated_attention": {"us": round(ungated, 2), "tflops": round(full_flops / ungated / 1e6, 1),
                               "frac_measured_bf16": round(full_flops / ungated / 1e6 / _peaks()["bf16"], 4)},
         "speedup_vs_ungated_attention": round(ungated / gated_total, 2),
+        "upper_stack": stack,
         "attention_backward": {"us": round(bwd_us, 2),
                                "tflops": round(kept_flops / bwd_us / 1e6, 1),
                                "frac_measured_bf16": round(kept_flops / bwd_us / 1e6 / _peaks()["bf16"], 4),
