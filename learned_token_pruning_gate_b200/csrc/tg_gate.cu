@@ -287,8 +287,8 @@ struct Gate2Layout {
   __host__ __device__ Gate2Layout(int dg) {
     a_box = kBM * kBK * 2;                             // 128 rows x 64 cols
     b_box = static_cast<uint32_t>(dg / 2) * kBK * 2;   // dg/2 rows x 64 cols
-    a_bytes = 2 * a_box;
-    stage_bytes = a_bytes + 2 * b_box;
+    a_bytes = (kBK2 / kBK) * a_box;
+    stage_bytes = a_bytes + (kBK2 / kBK) * b_box;
     bars_off = kStages2 * stage_bytes;
     misc_off = bars_off + 24 * 8;
     b1_off = misc_off + 16;
@@ -359,10 +359,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             break;
           const uint32_t sa = smem_u32(smem + stage * L.stage_bytes);
           if (leader) mbar_arrive_expect_tx(bar(stage), 2 * L.stage_bytes);
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < kBK2 / kBK; ++c)
             tma_load_2d_pair(sa + c * L.a_box, &tm_h, kb * kBK2 + c * kBK,
                              tile * 2 * kBM + rank * kBM, leader_bar(stage), pol_stream);
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < kBK2 / kBK; ++c)
             tma_load_2d_pair(sa + L.a_bytes + c * L.b_box, &tm_w, kb * kBK2 + c * kBK,
                              rank * (p.dg / 2), leader_bar(stage), pol_keep);
           if (++stage == kStages2) {
