@@ -380,16 +380,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             nph ^= 1;
           }
           const bool more = j + 1 < n_kv;
-          // head a: P_a(j) V_j, then S_a(j+1)
+          // head a: P_a(j) V_j, then S_a(j+1); the tiles are waited for first, so once
+          // P_a arrives both groups of MMAs issue back to back
+          if (!(ok = wt(v_full(rs), rph))) break;
+          if (more && !(ok = wt(k_full(ns), nph))) break;
           if (!(ok = wt(bar(kPFull + 0), p_waits[0]++ & 1))) break;
           if (j == 0 && !(ok = wt(bar(kOFree + 0), (of_waits[0]++ & 1) ^ 1))) break;
-          if (!(ok = wt(v_full(rs), rph))) break;
           tc_fence_after();
           issue_pv(0, rs, j > 0);
           if (!more) umma_commit(bar(kOFull + 0));
           if (more) {
-            if (!(ok = wt(k_full(ns), nph))) break;
-            tc_fence_after();
             issue_s(0, ns, (tile_base + j + 1) & 1);
             if (!it.has_b && j + 2 == n_kv) umma_commit(bar(kQEmpty));
           }
