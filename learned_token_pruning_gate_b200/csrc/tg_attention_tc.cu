@@ -991,9 +991,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (n_kv <= 2) commit_both(kPQEmpty);
         for (int j = 0; j < n_kv; ++j) {
           const int bf = j & 1;
+          // the tiles first, so once P(j) arrives P.V and the next Q.K^T issue back to back
+          if (!(ok = mbar_wait(bar(kPVFull + vs), vph, abort_flag, p.status, kDevTimeoutAttn))) break;
+          if (j + 2 < n_kv &&
+              !(ok = mbar_wait(bar(kPKFull + ks), kph, abort_flag, p.status, kDevTimeoutAttn)))
+            break;
           if (!wait_slot(kPPFull + bf)) break;
           if (j == 0 && !wait_slot(kPOFree)) break;
-          if (!(ok = mbar_wait(bar(kPVFull + vs), vph, abort_flag, p.status, kDevTimeoutAttn))) break;
           tc_fence_after();
           const uint64_t dv = dv0 + ((vs * L::kVStage) >> 4);
           // P(j) V_j into O_bf: the softmax warpgroup of this parity owns both
@@ -1008,9 +1012,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             vph ^= 1;
           }
           if (j + 2 < n_kv) {
-            if (!(ok = mbar_wait(bar(kPKFull + ks), kph, abort_flag, p.status, kDevTimeoutAttn)))
-              break;
-            tc_fence_after();
             issue_s(bf, ks);  // P(j) in this buffer was read by the P.V above: in order
             commit_both(kPSFull + bf);
             commit_both(kPKEmpty + ks);
