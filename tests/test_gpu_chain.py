@@ -116,3 +116,24 @@ def test_chain_edge_cases(oracle):
     assert ok
     if ndiff == 0:
         assert_close("out", host_f32(g["out"]), ref["out"], *ATTN_BF16)
+
+
+def test_chain_maximum_batch(oracle):
+    """TG_MAX_BATCH prompts through the whole chain (small model shape)."""
+    rng = np.random.default_rng(91)
+    B = tg.MAX_BATCH
+    seq = rng.integers(1, 400, size=B)
+    seq[::23] = 1
+    qn = np.minimum(seq, rng.integers(0, 40, size=B))
+    bud = rng.integers(0, 200, size=B)
+    w = gen.Workload("max_batch", tuple(int(x) for x in seq), tuple(int(x) for x in qn),
+                     tuple(int(x) for x in bud), 128, 32, 4, 2, 64, "bf16", 0, 92)
+    inp = gen.make_inputs(w)
+    g = _run_gpu(inp)
+    ref = _oracle_chain(oracle, inp)
+    assert_close("z", g["z"].cpu().numpy(), ref["z"], GATE_ATOL, 0.0)
+    ok, ndiff = kept_set_agrees(g["kept_idx"].cpu().numpy(), ref["kept"], ref["z"], inp.cu_seqlens,
+                                inp.doc_begin, inp.doc_end, inp.budget)
+    assert ok
+    if ndiff == 0:
+        assert_close("out", host_f32(g["out"]), ref["out"], *ATTN_BF16)

@@ -175,3 +175,29 @@ def test_topk_budget_sweep_bit_exact(oracle, lens):
         ref, ref_cu = oracle.topk_select(z, cu, s, e, k)
         assert ck.cpu().numpy().tolist() == ref_cu.tolist() == host.tolist()
         np.testing.assert_array_equal(kk.cpu().numpy(), ref)
+
+
+def test_topk_maximum_batch(oracle):
+    """TG_MAX_BATCH prompts in one launch, empty and one-token prompts among them."""
+    rng = np.random.default_rng(77)
+    B = tg.MAX_BATCH
+    lens = rng.integers(0, 700, size=B)
+    lens[::17] = 0
+    lens[5::19] = 1
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q = np.minimum(lens, rng.integers(0, 64, size=B))
+    s = np.zeros(B, np.int32)
+    e = (lens - q).astype(np.int32)
+    k = rng.integers(0, 300, size=B).astype(np.int32)
+    z = gen.random_scores(int(cu[-1]), seed=78)
+    _topk_both(oracle, z, cu, s, e, k)
+
+
+def test_topk_longest_prompt(oracle):
+    """The longest prompt the cluster holds: 8 CTAs x 45056 keys; one more is refused."""
+    n = 8 * 45056
+    z = gen.random_scores(n, seed=79)
+    _topk_both(oracle, z, [0, n], [0], [n - 512], [n // 8])
+    z2 = torch.from_numpy(gen.random_scores(n + 1, seed=80)).cuda()
+    with pytest.raises(tg.TokenGateError, match="TG_ERR_UNSUPPORTED.*exceeds"):
+        tg.topk_select(z2, [0, n + 1], [0], [n], [1000])
