@@ -7,9 +7,12 @@
 // the kept indices and loads every tensor's row of the batch, warps 2-7 rotate
 // the q/k heads in place (RoPE) and write the bias term (two groups of three
 // warps taking alternate batches, so two batches rotate at once), warp 1 stores the rows
-// back with bulk shared->global copies.  Bytes in flight are bounded by shared
-// memory (4 x 48 KB per SM), not by registers, so a handful of threads keep
-// the HBM busy.
+// back with bulk shared->global copies.  A stage holds each tensor's rows of the
+// batch back to back; the compacted rows of a batch are consecutive in every
+// output, so each tensor leaves in one store (the copy engine is bound by its
+// number of operations more than by bytes for rows of a few KB).  Bytes in flight
+// are bounded by shared memory (4 x 48 KB per SM), not by registers, so a handful
+// of threads keep the HBM busy.
 //
 // Fallback (rows wider than a stage): one warp moves one (kept row, tensor)
 // pair with 16-byte vector loads and stores.  Rows that carry attention heads are rotated by RoPE at their
@@ -229,7 +232,7 @@ struct BulkParams {
   const uint8_t* src[TG_MAX_GATHER_TENSORS];
   uint8_t* dst[TG_MAX_GATHER_TENSORS];
   int32_t row_bytes[TG_MAX_GATHER_TENSORS];
-  int32_t row_off[TG_MAX_GATHER_TENSORS];  // offset of the tensor's row inside a batch row
+  int32_t row_off[TG_MAX_GATHER_TENSORS];  // bytes of the tensors before this one in a kept row
   int32_t rope_heads[TG_MAX_GATHER_TENSORS];
   // RoPE angle of position pos, dim i: pos * theta^(-2i/d) radians, kept as a
   // fraction of a turn in 0.64 fixed point (evaluated on the host in fp64): the
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) gather_bulk_kernel(const __gr
           if (sm.src_row[s][r] < 0) continue;
           const int64_t row = sm.src_row[s][r];
           for (int t = 0; t < p.n_tensors; ++t)
-            bulk_g2s(base + r * p.row_total + p.row_off[t], p.src[t] + row * p.row_bytes[t],
+            bulk_g2s(base + p.rows * p.row_off[t] + r * p.row_bytes[t], p.src[t] + row * p.row_bytes[t],
                      p.row_bytes[t], fb);
         }
       }
@@ -364,12 +367,23 @@ __global__ void __launch_bounds__(kBulkThreads, 1) gather_bulk_kernel(const __gr
         const int i0 = batch * p.rows;
         const int n = min(p.rows, p.m_total - i0);
         const uint32_t base = smem_u32(sm.stage[s]);
-        for (int r = 0; r < n; ++r) {
-          if (sm.src_row[s][r] < 0) continue;
-          const int64_t i = i0 + r;
+        // a stage holds each tensor's rows of the batch back to back, and the
+        // compacted rows are consecutive: one store per tensor (per row only when
+        // an invalid index left a row unloaded)
+        bool all_valid = true;
+        for (int r = 0; r < n; ++r) all_valid &= sm.src_row[s][r] >= 0;
+        if (all_valid) {
           for (int t = 0; t < p.n_tensors; ++t)
-            bulk_s2g(p.dst[t] + i * p.row_bytes[t], base + r * p.row_total + p.row_off[t],
-                     p.row_bytes[t]);
+            bulk_s2g(p.dst[t] + static_cast<int64_t>(i0) * p.row_bytes[t],
+                     base + p.rows * p.row_off[t], n * p.row_bytes[t]);
+        } else {
+          for (int r = 0; r < n; ++r) {
+            if (sm.src_row[s][r] < 0) continue;
+            const int64_t i = i0 + r;
+            for (int t = 0; t < p.n_tensors; ++t)
+              bulk_s2g(p.dst[t] + i * p.row_bytes[t], base + p.rows * p.row_off[t] + r * p.row_bytes[t],
+                       p.row_bytes[t]);
+          }
         }
         bulk_commit();
         // hand the stage back as soon as these stores have read it
@@ -429,7 +443,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) gather_bulk_kernel(const __gr
           for (int e = 0; e < VE; ++e) w[e] = cs_buf[r * half + cvec * VE + e];
           for (int t = 0; t < p.n_tensors; ++t) {
             const int nh = p.rope_heads[t];
-            uint4* base = reinterpret_cast<uint4*>(sm.stage[s] + r * p.row_total + p.row_off[t]) + cvec;
+            uint4* base = reinterpret_cast<uint4*>(sm.stage[s] + p.rows * p.row_off[t] + r * p.row_bytes[t]) + cvec;
             const int hstep = p.head_dim / VE;  // vectors per head
             for (int h = hg; h < nh; h += 2 * nhg) {
               const bool two = h + nhg < nh;
