@@ -536,6 +536,25 @@ def run_extras(args):
                  "note": "Qwen3-1.7B-shaped (d 2048, 16/8 x 128, MLP 6144), random init; GEMMs "
                          "cuBLAS, other steps libtokengate"}
         del st_, xs, sl
+    # a Gated DeltaNet layer of a hybrid backbone over the same kept rows: the gated
+    # delta rule, sequential over each prompt's rows, fp32 state per (prompt, head)
+    dcu, dq, dkk, dvv, dla, dbeta = gen.delta_inputs(w.kept_lengths(), w.n_q_heads, w.head_dim,
+                                                     w.seed, w.dtype)
+    dq, dkk, dvv, dla, dbeta = (d(x) for x in (dq, dkk, dvv, dla, dbeta))
+    d_out = torch.empty_like(dvv)
+    d_state = torch.empty((len(dcu) - 1, w.n_q_heads, w.head_dim, w.head_dim), dtype=torch.float32,
+                          device=dev)
+    delta_us = timed(lambda: tg.gated_delta_scan(dq, dkk, dvv, dcu, dla, dbeta, out=d_out,
+                                                 state=d_state), 10)
+    # per row and head: S k, the rank-1 update (scale + FMA) and S q over d x d
+    delta_flops = 7.0 * w.head_dim ** 2 * w.n_q_heads * Mk
+    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # FMA lanes x 2 flop x max SM clock, TFLOP/s
+    delta = {"us": round(delta_us, 2), "rows_per_s": round(Mk / delta_us * 1e6),
+             "tflops_fp32": round(delta_flops / delta_us / 1e6, 3),
+             "frac_alu_nominal": round(delta_flops / delta_us / 1e6 / fp32_peak, 4),
+             "heads": w.n_q_heads, "head_dim": w.head_dim,
+             "note": "recurrent form: latency of one row's update chain x rows per prompt"}
+    del dq, dkk, dvv, dla, dbeta, d_out, d_state
     del layer, o_f, lse_f, dout, bws
     torch.cuda.synchronize()
     # ungated: every token of every prompt attends causally, no bias (the layer without a gate)
@@ -566,6 +585,7 @@ def run_extras(args):
                               "frac_measured_bf16": round(full_flops / ungated / 1e6 / _peaks()["bf16"], 4)},
         "speedup_vs_ungated_attention": round(ungated / gated_total, 2),
         "upper_stack": stack,
+        "delta_scan": delta,
         "attention_backward": {"us": round(bwd_us, 2),
                                "tflops": round(kept_flops / bwd_us / 1e6, 1),
                                "frac_measured_bf16": round(kept_flops / bwd_us / 1e6 / _peaks()["bf16"], 4),

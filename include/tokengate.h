@@ -370,6 +370,31 @@ TG_API tg_status tg_qkv_rope_emit(const void* qkv, tg_dtype dtype, int32_t batch
 TG_API tg_status tg_swiglu(const void* gate_up, void* out, tg_dtype dtype, int64_t rows,
                            int32_t inter, tg_stream_t stream);
 
+/*
+ * tg_gated_delta_scan: a Gated DeltaNet (linear-attention) layer of a hybrid
+ * backbone above the gate, over each prompt's kept rows only.  TokenGate prunes
+ * these layers as well as the attention layers (lucasainews.com, "성능 결과",
+ * with its comparison table; lefilia.fr, body; the abstract's "hybrid-attention
+ * models").  The pages do not write the layer out; this is the published gated
+ * delta rule (Gated DeltaNet), with no gate bias (the bias acts on attention
+ * logits) and a zero initial state.  Per prompt b and head h, over the kept rows
+ * t of b in order:
+ *   k^_t = k_t / sqrt(|k_t|^2 + eps),   q^_t = q_t / sqrt(|q_t|^2 + eps) / sqrt(head_dim)
+ *   S_t  = alpha_t S_{t-1} + beta_t (v_t - alpha_t S_{t-1} k^_t) k^_t^T,  alpha_t = exp(log_alpha_t)
+ *   out_t = S_t q^_t
+ *   q, k, v        [M, n_heads, head_dim] (device, dtype, 16-byte aligned), M = cu_kept_h[batch]
+ *   log_alpha,beta [M, n_heads] fp32 (log_alpha <= 0 keeps the state bounded; -inf is alpha = 0)
+ *   cu_kept_h      [batch + 1] host array (prefix sums of the kept rows per prompt)
+ *   out            [M, n_heads, head_dim] (dtype)
+ *   state_out      [batch, n_heads, head_dim (v), head_dim (k)] fp32: S after each prompt's
+ *                  last row (zero for a prompt with no rows); NULL to skip
+ *   head_dim 64 or 128 (else TG_ERR_UNSUPPORTED); state kept in fp32.
+ */
+TG_API tg_status tg_gated_delta_scan(const void* q, const void* k, const void* v, tg_dtype dtype,
+                                     const float* log_alpha, const float* beta, int32_t batch,
+                                     const int32_t* cu_kept_h, int32_t n_heads, int32_t head_dim,
+                                     float eps, void* out, float* state_out, tg_stream_t stream);
+
 /* Workspace bytes tg_gated_attention_backward needs for this batch (host-only). */
 TG_API tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,
                                                        int32_t n_q_heads, size_t* bytes_out);

@@ -25,7 +25,7 @@ __all__ = [
     "library", "kept_offsets", "gate_score", "topk_select", "compact_gather", "gated_attention",
     "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
     "attention_kernel", "topk_select_multi", "random_select", "gated_attention_backward",
-    "attention_backward_workspace_bytes", "rmsnorm", "qkv_rope_emit", "swiglu",
+    "attention_backward_workspace_bytes", "rmsnorm", "qkv_rope_emit", "swiglu", "gated_delta_scan",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = (
     "tg_gated_attention", "tg_attention_workspace_bytes", "tg_attention_kernel",
     "tg_gated_attention_noalloc", "tg_topk_select_multi", "tg_random_select",
     "tg_gated_attention_backward", "tg_attention_backward_workspace_bytes", "tg_rmsnorm",
-    "tg_qkv_rope_emit", "tg_swiglu",
+    "tg_qkv_rope_emit", "tg_swiglu", "tg_gated_delta_scan",
 )
 MAX_BUDGETS = 8
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
@@ -108,6 +108,8 @@ def library():
     L.tg_qkv_rope_emit.argtypes = [_vp, ctypes.c_int, _i32, _i32p, _i32p, _vp, _i32, _i32, _i32,
                                    _vp, _vp, _f32, ctypes.c_double, _vp, _vp, _vp, _vp]
     L.tg_swiglu.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i32, _vp]
+    L.tg_gated_delta_scan.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _i32, _i32p, _i32, _i32,
+                                      _f32, _vp, _vp, _vp]
     for name in EXPORTED_SYMBOLS:
         if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -414,6 +416,25 @@ def swiglu(gate_up, out=None):
     _check("tg_swiglu", library().tg_swiglu(_ptr(gate_up), _ptr(out), _dtype_code(gate_up), rows,
                                             two // 2, _stream(gate_up.device)))
     return out
+
+
+def gated_delta_scan(q, k, v, cu_kept_host, log_alpha, beta, eps=1e-6, out=None, state=None,
+                     want_state=True):
+    """Gated delta rule over each prompt's kept rows (a Gated DeltaNet layer above the
+    gate): q, k, v [M, H, d] (d 64 or 128), log_alpha, beta [M, H] fp32.  Returns
+    (o [M, H, d], state [B, H, d, d] fp32 or None)."""
+    _need_cuda(q, k, v, log_alpha, beta)
+    M, H, d = q.shape
+    ck, ck_p = _host_i32(cu_kept_host)
+    B = len(ck) - 1
+    if out is None:
+        out = torch.empty_like(v)
+    if state is None and want_state:
+        state = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    _check("tg_gated_delta_scan", library().tg_gated_delta_scan(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), B, ck_p, H, d,
+        float(eps), _ptr(out), _ptr(state) if state is not None else None, _stream(q.device)))
+    return out, state
 
 
 def gated_prefill(h, q, k, v, W1, b1, w2, b2, gain, temp, cu_seqlens, doc_begin, doc_end,

@@ -471,6 +471,29 @@ tg_status tg_swiglu(const void* gate_up, void* out, tg_dtype dtype, int64_t rows
   return launch_swiglu(gate_up, out, dtype, rows, inter, reinterpret_cast<cudaStream_t>(stream));
 }
 
+tg_status tg_gated_delta_scan(const void* q, const void* k, const void* v, tg_dtype dtype,
+                              const float* log_alpha, const float* beta, int32_t batch,
+                              const int32_t* cu_kept_h, int32_t n_heads, int32_t head_dim, float eps,
+                              void* out, float* state_out, tg_stream_t stream) {
+  if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
+  PromptTable t;
+  int max_len = 0;
+  tg_status r = build_kept_table(batch, cu_kept_h, &t, &max_len);
+  if (r != TG_OK) return r;
+  if (n_heads <= 0) return set_error(TG_ERR_SHAPE, "n_heads=%d", n_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(TG_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", head_dim);
+  if (!(eps >= 0.0f)) return set_error(TG_ERR_INVALID_ARG, "eps must be >= 0");
+  if (batch == 0 || (t.kept_start[batch] == 0 && !state_out)) return TG_OK;
+  if (t.kept_start[batch] > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+    return set_error(TG_ERR_INVALID_ARG, "null pointer");
+  for (const void* ptr : {q, k, v, static_cast<const void*>(state_out)})
+    if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0)
+      return set_error(TG_ERR_ALIGNMENT, "q, k, v and state_out must be 16-byte aligned");
+  return launch_delta_scan(q, k, v, dtype, log_alpha, beta, t, n_heads, head_dim, eps, out, state_out,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
 tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,
                                                 int32_t n_q_heads, size_t* bytes_out) {
   if (!bytes_out) return set_error(TG_ERR_INVALID_ARG, "bytes_out is NULL");

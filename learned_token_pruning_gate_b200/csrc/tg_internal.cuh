@@ -74,6 +74,9 @@ tg_status launch_rmsnorm(const void* x, const void* w, void* y, tg_dtype dt, int
 tg_status launch_qkv_emit(const void* qkv, tg_dtype dt, const PromptTable& pt, const int32_t* kept_idx,
                           int hq, int hkv, int dh, const void* w_qn, const void* w_kn, float eps,
                           double theta, void* q_out, void* k_out, void* v_out, cudaStream_t st);
+tg_status launch_delta_scan(const void* q, const void* k, const void* v, tg_dtype dt,
+                            const float* log_alpha, const float* beta, const PromptTable& pt, int heads,
+                            int head_dim, float eps, void* out, float* state, cudaStream_t st);
 tg_status launch_swiglu(const void* gu, void* h, tg_dtype dt, int64_t rows, int inter,
                         cudaStream_t st);
 // Workspace the tensor-core attention uses to split long items on this device (0 = none).

@@ -235,3 +235,20 @@ def attention_inputs(M_list, Hq, Hkv, dh, seed, dtype="bf16", bias=True):
     gain = torch.from_numpy(rng.uniform(0.0, 1.0, Hq).astype(np.float32))
     temp = torch.from_numpy(rng.uniform(0.8, 1.2, Hq).astype(np.float32))
     return cu, q, k, v, ls, gain, temp
+
+
+def delta_inputs(M_list, H, d, seed, dtype="bf16", decay=0.1):
+    """Kept-row inputs of a gated-delta-rule layer: q, k, v [M, H, d] ~ N(0, 1) in
+    `dtype`; log_alpha = -U(0, decay) (per-token decays alpha in (e^-decay, 1]);
+    beta = sigmoid(N(0, 1)) [M, H] fp32."""
+    rng = np.random.Generator(np.random.Philox(seed))
+    dt = _tdtype(dtype)
+    M = int(sum(M_list))
+    cu = np.zeros(len(M_list) + 1, np.int32)
+    cu[1:] = np.cumsum(M_list)
+    q = torch.from_numpy(_normal(rng, (M, H, d))).to(dt)
+    k = torch.from_numpy(_normal(rng, (M, H, d))).to(dt)
+    v = torch.from_numpy(_normal(rng, (M, H, d))).to(dt)
+    la = torch.from_numpy(-rng.uniform(0.0, decay, (M, H)).astype(np.float32))
+    beta = torch.from_numpy((1.0 / (1.0 + np.exp(-_normal(rng, (M, H))))).astype(np.float32))
+    return cu, q, k, v, la, beta

@@ -280,3 +280,29 @@ def test_attention_backward_validation(L):
     _, ck0 = _arr([0, 0])
     assert b(None, None, None, 0, 1, ck0, 16, 8, 128, None, None, None, None, None, None, None,
              None, None, None, None, 0, 0, None) == OK
+
+
+def test_delta_scan_validation(L):
+    """The gated delta scan rejects bad arguments before launching anything."""
+    _, ck = _arr([0, 40, 90])
+    f = L.tg_gated_delta_scan
+
+    def call(dtype=0, batch=2, cu=ck, heads=4, d=128, eps=1e-6, q=FAKE, la=FAKE, state=FAKE):
+        return f(q, FAKE, FAKE, dtype, la, FAKE, batch, cu, heads, d, eps, FAKE, state, None)
+
+    assert call(dtype=5) == DTYPE
+    assert call(heads=0) == SHAPE
+    assert call(d=96) == UNSUP
+    assert call(eps=-1.0) == INVALID
+    assert call(eps=float("nan")) == INVALID
+    assert call(q=None) == INVALID
+    assert call(la=None) == INVALID
+    assert call(q=FAKE_ODD) == ALIGN
+    assert call(state=FAKE_ODD) == ALIGN
+    assert call(batch=tg.MAX_BATCH + 1, cu=_arr(list(range(tg.MAX_BATCH + 2)))[1]) == UNSUP
+    assert call(cu=_arr([0, 50, 40])[1]) == INVALID  # a prompt with a negative count
+    assert call(cu=_arr([3, 50, 90])[1]) == INVALID
+    # nothing kept and no state wanted: nothing to do
+    _, ck0 = _arr([0, 0])
+    assert f(None, None, None, 0, None, None, 1, ck0, 4, 64, 1e-6, None, None, None) == OK
+    assert f(None, None, None, 0, None, None, 0, ck0, 4, 64, 1e-6, None, None, None) == OK
