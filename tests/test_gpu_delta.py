@@ -95,3 +95,35 @@ def test_delta_scan_rejects_unsupported_head_dim():
     with pytest.raises(tg.TokenGateError, match="TG_ERR_UNSUPPORTED"):
         tg.gated_delta_scan(x, x, x, [0, 4], torch.zeros(4, 1, device="cuda"),
                             torch.zeros(4, 1, device="cuda"))
+
+
+def test_delta_scan_maximum_batch():
+    """TG_MAX_BATCH prompts of ragged lengths (0 to 40 rows): every prompt's state
+    starts from zero and ends where the oracle says."""
+    rng = np.random.default_rng(4)
+    lens = [int(x) for x in rng.integers(0, 41, tg.MAX_BATCH)]
+    o, s, ro, rs = _run(lens, 2, 64, "fp32", seed=12, decay=0.3)
+    assert_close("out", o, ro, 1e-4, 1e-3)
+    assert_close("state", s, rs, 1e-4, 1e-3)
+
+
+def test_delta_scan_over_the_gated_layers_kept_rows():
+    """The layer consumes what the gated layer produces: the compacted q, k, v of a
+    gated prefill (kept rows only, RoPE applied) as its inputs."""
+    w = gen.scaled(gen.WORKLOADS["qwen_16k"], 8, name="delta_chain")
+    inp = gen.make_inputs(w)
+    r = tg.gated_prefill(*(dev(x) for x in (inp.h, inp.q, inp.k, inp.v, inp.W1, inp.b1, inp.w2)),
+                         inp.b2, dev(inp.gain), dev(inp.temp), inp.cu_seqlens, inp.doc_begin,
+                         inp.doc_end, inp.budget, rope_theta=w.rope_theta)
+    ck = r["cu_kept_host"]
+    M = int(ck[-1])
+    H = r["k"].shape[1]
+    rng = np.random.default_rng(5)
+    la = torch.from_numpy(-rng.uniform(0.0, 0.1, (M, H)).astype(np.float32))
+    beta = torch.from_numpy(rng.uniform(0.0, 1.0, (M, H)).astype(np.float32))
+    q = r["q"][:, :H].contiguous()  # one query head per state head
+    o, s = tg.gated_delta_scan(q, r["k"], r["v"], ck, dev(la), dev(beta))
+    torch.cuda.synchronize()
+    ro, rs = do.scan(host_f32(q), host_f32(r["k"]), host_f32(r["v"]), la.numpy(), beta.numpy(), ck)
+    assert_close("out", host_f32(o), ro, 2e-3, 2.0 ** -7)
+    assert_close("state", host_f32(s), rs, 1e-4, 1e-3)
