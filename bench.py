@@ -422,10 +422,19 @@ def run_ncu_case(args):
         bwd = lambda: tg.gated_attention_backward(  # noqa: E731
             layer.q_c, layer.k_c, layer.v_c, layer.cu_kept_host, layer.logsig, layer.gain,
             layer.temp, o, lse, dout)
+    delta = None
+    if args.delta:
+        # a gated-delta-rule layer over the kept rows (one state head per query head)
+        _, dq, dkk, dvv, dla, dbeta = gen.delta_inputs([layer.M], w.n_q_heads, w.head_dim, w.seed,
+                                                       w.dtype)
+        dq, dkk, dvv, dla, dbeta = (d(x) for x in (dq, dkk, dvv, dla, dbeta))
+        delta = lambda: tg.gated_delta_scan(dq, dkk, dvv, layer.cu_kept_host, dla, dbeta)  # noqa: E731
     for _ in range(args.steps):
         layer.run()
         if bwd:
             bwd()
+        if delta:
+            delta()
     torch.cuda.synchronize()
     if tg.device_status() != 0:
         raise SystemExit("a kernel reported a timed-out wait")
@@ -621,6 +630,8 @@ def main():
                     help="print bias overhead, ungated full-N attention and memory figures")
     ap.add_argument("--ncu-case", action="store_true",
                     help="untimed: run --steps plain steps of the workload (profiling)")
+    ap.add_argument("--delta", action="store_true",
+                    help="with --ncu-case: also run the gated-delta-rule scan over the kept rows")
     ap.add_argument("--backward", action="store_true",
                     help="with --ncu-case: also run the attention backward after each step")
     args = ap.parse_args()
