@@ -423,9 +423,21 @@ def gated_delta_scan(q, k, v, cu_kept_host, log_alpha, beta, eps=1e-6, out=None,
     """Gated delta rule over each prompt's kept rows (a Gated DeltaNet layer above the
     gate): q, k, v [M, H, d] (d 64 or 128), log_alpha, beta [M, H] fp32.  Returns
     (o [M, H, d], state [B, H, d, d] fp32 or None)."""
-    _need_cuda(q, k, v, log_alpha, beta)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError(f"q, k, v must share one [M, H, d] shape: {tuple(q.shape)}, "
+                         f"{tuple(k.shape)}, {tuple(v.shape)}")
     M, H, d = q.shape
+    if tuple(log_alpha.shape) != (M, H) or tuple(beta.shape) != (M, H):
+        raise ValueError(f"log_alpha and beta must be [M, H] = {(M, H)}")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise ValueError("log_alpha and beta must be float32")
+    for t in (q, k, v, log_alpha, beta):
+        if not t.is_contiguous():
+            raise ValueError("gated_delta_scan takes contiguous tensors")
+    _need_cuda(q, k, v, log_alpha, beta)
     ck, ck_p = _host_i32(cu_kept_host)
+    if int(ck[-1]) != M:
+        raise ValueError(f"cu_kept_host ends at {int(ck[-1])}, q has {M} rows")
     B = len(ck) - 1
     if out is None:
         out = torch.empty_like(v)

@@ -484,6 +484,9 @@ tg_status tg_gated_delta_scan(const void* q, const void* k, const void* v, tg_dt
   if (head_dim != 64 && head_dim != 128)
     return set_error(TG_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", head_dim);
   if (!(eps >= 0.0f)) return set_error(TG_ERR_INVALID_ARG, "eps must be >= 0");
+  if (static_cast<int64_t>(batch) * n_heads * (head_dim / 32) > INT32_MAX)
+    return set_error(TG_ERR_UNSUPPORTED, "batch x n_heads = %lld state slices exceed one launch",
+                     static_cast<long long>(batch) * n_heads);
   if (batch == 0 || (t.kept_start[batch] == 0 && !state_out)) return TG_OK;
   if (t.kept_start[batch] > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
     return set_error(TG_ERR_INVALID_ARG, "null pointer");

@@ -306,3 +306,27 @@ def test_delta_scan_validation(L):
     _, ck0 = _arr([0, 0])
     assert f(None, None, None, 0, None, None, 1, ck0, 4, 64, 1e-6, None, None, None) == OK
     assert f(None, None, None, 0, None, None, 0, ck0, 4, 64, 1e-6, None, None, None) == OK
+
+
+def test_delta_scan_launch_size_bound(L):
+    """batch x heads x state slices beyond one launch's blocks is rejected."""
+    cu, ck = _arr([0] * (tg.MAX_BATCH + 1))
+    heads = (2 ** 31) // (tg.MAX_BATCH * 4) + 1
+    assert L.tg_gated_delta_scan(None, None, None, 0, None, None, tg.MAX_BATCH, ck, heads, 128, 1e-6,
+                                 None, FAKE, None) == UNSUP
+
+
+def test_delta_scan_wrapper_rejects_mismatched_shapes():
+    """The Python binding checks shapes before anything reaches the library."""
+    import torch
+
+    x = torch.zeros(6, 2, 64)
+    a = torch.zeros(6, 2)
+    with pytest.raises(ValueError, match="share one"):
+        tg.gated_delta_scan(x, torch.zeros(6, 2, 32), x, [0, 6], a, a)
+    with pytest.raises(ValueError, match=r"\[M, H\]"):
+        tg.gated_delta_scan(x, x, x, [0, 6], torch.zeros(6, 3), a)
+    with pytest.raises(ValueError, match="float32"):
+        tg.gated_delta_scan(x, x, x, [0, 6], a.double(), a)
+    with pytest.raises(ValueError, match="CUDA"):
+        tg.gated_delta_scan(x, x, x, [0, 6], a, a)

@@ -84,3 +84,4 @@ def test_prompts_are_independent():
         ob, sb = delta.scan(q[r0:r1], k[r0:r1], v[r0:r1], la[r0:r1], be[r0:r1], [0, r1 - r0])
         assert np.array_equal(o[r0:r1], ob)
         assert np.array_equal(state[b], sb[0])
+
