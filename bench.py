@@ -280,12 +280,7 @@ def run_gpu(args):
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "prompts_per_gpu": w.batch,
-                   "seq_len": list(w.seqlens), "question": list(w.question),
-                   "budget_K": list(w.budgets), "kept_M": w.kept_lengths(),
-                   "d_model": w.d_model, "gate": f"{w.d_model}->{w.d_hidden}->1",
-                   "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv x {w.head_dim}",
-                   "parallelism": f"replicas x{world} (independent prompts, no collective)",
+        "config": {**_workload_config(args.workload, w, world),
                    "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
                    "timing": "CUDA events per step around a CUDA-graph replay of the 4 launches"},
         "gpu_launches": 4 * K,
@@ -367,6 +362,15 @@ def cpu_baseline(inp, seconds=15.0, repeats=1):
             "seconds_per_step_extrapolated": total}
 
 
+def _workload_config(name, w, world):
+    """The workload keys of the bench line's config (shared by both arms)."""
+    return {"workload": name, "prompts_per_gpu": w.batch, "seq_len": list(w.seqlens),
+            "question": list(w.question), "budget_K": list(w.budgets), "kept_M": w.kept_lengths(),
+            "d_model": w.d_model, "gate": f"{w.d_model}->{w.d_hidden}->1",
+            "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv x {w.head_dim}",
+            "parallelism": f"replicas x{world} (independent prompts, no collective)"}
+
+
 def run_reference(args):
     """Reference arm: the CPU oracle on this workload, on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
@@ -389,11 +393,14 @@ def run_reference(args):
     cb = dict(vals[-1])
     cb["value"] = value
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 0,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "device": "host cores",
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.total_tokens / value * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": args.workload, "seq_len": list(w.seqlens),
-                                        "budget_K": list(w.budgets)},
+        "data": "synthetic",
+        "config": {**_workload_config(args.workload, w, int(os.environ.get("WORLD_SIZE", args.gpus))),
+                   "timing": "wall clock of the fp64 oracle on rank 0's host cores; each step a "
+                             "bounded sample of the workload, extrapolated to all of it"},
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
