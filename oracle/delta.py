@@ -25,6 +25,8 @@ independent statement of the same function used to pin it: unrolling the
 recurrence gives S_t = sum_{s<=t} (g_t / g_s) u_s k^_s^T with g_t = prod_{r<=t}
 alpha_r and u_t = beta_t (v_t - sum_{s<t} (g_t / g_s) (k^_s . k^_t) u_s), a unit
 lower-triangular system (I + A) U = diag(beta) V solved with a library solver.
+``scan_chunked`` states the same function chunk by chunk (the form a parallel kernel
+takes: the state before a chunk enters every row's equation of that chunk).
 """
 from __future__ import annotations
 
@@ -95,4 +97,41 @@ def scan_closed_form(q, k, v, log_alpha, beta, cu_kept, eps=1e-6):
             U = np.linalg.solve(np.eye(n) + A, be[r0:r1, h][:, None] * V)
             o[r0:r1, h] = (decay * (Q @ K.T)) @ U
             state[b, h] = (np.exp(lg[-1] - lg)[:, None] * U).T @ K
+    return o, state
+
+
+def scan_chunked(q, k, v, log_alpha, beta, cu_kept, chunk=16, eps=1e-6):
+    """The same outputs computed chunk by chunk, the form a parallel kernel takes:
+    with S_0 the state before a chunk and g_t = prod of alpha from the chunk's start,
+    u_t = beta_t (v_t - g_t S_0 k^_t - sum_{s<t} (g_t/g_s) (k^_s . k^_t) u_s) (a unit
+    lower-triangular solve), o_t = g_t S_0 q^_t + sum_{s<=t} (g_t/g_s) (k^_s . q^_t) u_s,
+    and the state after the chunk g_C S_0 + sum_s (g_C/g_s) u_s k^_s^T."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    la = np.asarray(log_alpha, np.float64)
+    be = np.asarray(beta, np.float64)
+    M, H, dk = q.shape
+    dv = v.shape[2]
+    qn = _normalise(q, eps) / np.sqrt(dk)
+    kn = _normalise(k, eps)
+    o = np.zeros((M, H, dv))
+    B = len(cu_kept) - 1
+    state = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dv, dk))
+            for c0 in range(int(cu_kept[b]), int(cu_kept[b + 1]), chunk):
+                c1 = min(c0 + chunk, int(cu_kept[b + 1]))
+                n = c1 - c0
+                K, Q, V, bt = kn[c0:c1, h], qn[c0:c1, h], v[c0:c1, h], be[c0:c1, h]
+                lg = np.cumsum(la[c0:c1, h])
+                g = np.exp(lg)
+                on_or_below = np.tril(np.ones((n, n), dtype=bool))
+                decay = np.exp(np.where(on_or_below, lg[:, None] - lg[None, :], -np.inf))
+                A = bt[:, None] * decay * (K @ K.T) * np.tril(np.ones((n, n)), -1)
+                U = np.linalg.solve(np.eye(n) + A, bt[:, None] * (V - g[:, None] * (K @ S.T)))
+                o[c0:c1, h] = g[:, None] * (Q @ S.T) + (decay * (Q @ K.T)) @ U
+                S = g[-1] * S + (np.exp(lg[-1] - lg)[:, None] * U).T @ K
+            state[b, h] = S
     return o, state

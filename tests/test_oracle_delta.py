@@ -85,3 +85,14 @@ def test_prompts_are_independent():
         assert np.array_equal(o[r0:r1], ob)
         assert np.array_equal(state[b], sb[0])
 
+
+
+@pytest.mark.parametrize("chunk", [1, 5, 16, 64])
+def test_chunked_form_equals_recurrence(chunk):
+    """The chunk-by-chunk statement (the form a parallel kernel takes) agrees with the
+    recurrence for chunks of one row, uneven chunks and chunks longer than a prompt."""
+    q, k, v, la, be, cu = _inputs([37, 0, 50, 1], decay=1.0, seed=7)
+    o1, s1 = delta.scan(q, k, v, la, be, cu)
+    o2, s2 = delta.scan_chunked(q, k, v, la, be, cu, chunk=chunk)
+    assert np.allclose(o1, o2, rtol=1e-10, atol=1e-12)
+    assert np.allclose(s1, s2, rtol=1e-10, atol=1e-12)
