@@ -388,7 +388,11 @@ TG_API tg_status tg_swiglu(const void* gate_up, void* out, tg_dtype dtype, int64
  *   out            [M, n_heads, head_dim] (dtype)
  *   state_out      [batch, n_heads, head_dim (v), head_dim (k)] fp32: S after each prompt's
  *                  last row (zero for a prompt with no rows); NULL to skip
- *   head_dim 64 or 128 (else TG_ERR_UNSUPPORTED); state kept in fp32.
+ *   head_dim 64 or 128 (else TG_ERR_UNSUPPORTED); state kept in fp32.  One CTA per 32 state
+ *   rows of a (prompt, head): batch x n_heads x head_dim / 32 above INT32_MAX is
+ *   TG_ERR_UNSUPPORTED.  Errors: TG_ERR_DTYPE, TG_ERR_SHAPE (n_heads <= 0),
+ *   TG_ERR_INVALID_ARG (cu_kept_h, eps < 0, null pointers with rows to process),
+ *   TG_ERR_ALIGNMENT; nothing is launched on an error.
  */
 TG_API tg_status tg_gated_delta_scan(const void* q, const void* k, const void* v, tg_dtype dtype,
                                      const float* log_alpha, const float* beta, int32_t batch,
