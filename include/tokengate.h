@@ -11,10 +11,14 @@
  * selection trainable, each kept token's score enters the attention logits above
  * the gate as a bias (the Mixture-of-Experts router trick) with a per-head
  * learned gain, and a per-head learned temperature corrects for each query
- * seeing fewer keys.  The four calls below are that forward pass, one call per
- * step:
+ * seeing fewer keys.  Four calls are that forward pass, one call per step:
  *
  *     tg_gate_score -> tg_topk_select -> tg_compact_gather -> tg_gated_attention
+ *
+ * Further calls serve the layers around it: budget sweeps and random-K selection,
+ * the backward of the gated attention (gradients of the log-gates, gains and
+ * temperatures), the element-wise steps of a stack of gated upper layers that
+ * emits a compacted KV cache, and a Gated DeltaNet layer over the kept rows.
  *
  * Conventions shared by every call
  *   - Device pointers point to memory on the current CUDA device; "host" arrays
