@@ -75,3 +75,21 @@ def test_backward_plants_a_mistake(seed):
                    for e in np.eye(len(t))])
     np.testing.assert_allclose(d_t, fd, atol=1e-7 * np.abs(fd).max())
     assert np.abs(d_t * t - fd).max() > 1e-3 * np.abs(fd).max()
+
+
+def test_loss_is_the_forward_inner_product(oracle):
+    """The loss that the finite differences differentiate is tied to the pinned
+    forward: L = sum(dout * out) with out from the oracle's gated attention (whose
+    own pins fix the bias sign, the temperature's place and the GQA map).  A
+    mistake in the loss's private attention row -- a flipped bias, the
+    temperature on the bias, a wrong kv head -- would keep the analytic and
+    numerical gradients consistent with each other, but not with this."""
+    q, k, v, cu, l, g, t, dout = _case([5, 9, 1, 12, 3], Hq=6, Hkv=2, dh=8, seed=11)
+    # the forward takes float32 log-gates, gains and temperatures: use values
+    # that float32 holds exactly, so both sides see the same numbers
+    l, g, t = (np.asarray(a, np.float32).astype(np.float64) for a in (l, g * 1.5, t * 1.4))
+    out, _ = oracle.gated_attention(q, k, v, cu, logsig=l, gain=g, temp=t)
+    terms = dout.astype(np.float64) * out
+    ref = float(terms.sum())
+    got = oracle.attention_loss(q, k, v, cu, l, g, t, dout)
+    assert abs(got - ref) <= 1e-12 * np.abs(terms).sum(), (got, ref)

@@ -10,6 +10,7 @@ import os
 import pytest
 
 import tests.test_oracle_attention as pa
+import tests.test_oracle_backward as pb
 import tests.test_oracle_gate_gather as pg
 import tests.test_oracle_topk as pt
 
@@ -41,6 +42,20 @@ MUTATIONS = [
     ("logsig_on_question", "out[i] = is_doc ? log_sigmoid((double)z[row]) : 0.0;",
      "out[i] = log_sigmoid((double)z[row]);",
      lambda o: pg.test_logsig_matches_torch_and_protects_question(o)),
+    # the attention row behind the backward's loss (tgo_attention_loss)
+    ("loss_bias_sign", "double lg = dot * scale + gain[h] * logsig[j];",
+     "double lg = dot * scale - gain[h] * logsig[j];",
+     lambda o: pb.test_loss_is_the_forward_inner_product(o)),
+    ("loss_temperature_on_bias", "double lg = dot * scale + gain[h] * logsig[j];",
+     "double lg = dot * scale + gain[h] * logsig[j] / temp[h];",
+     lambda o: pb.test_loss_is_the_forward_inner_product(o)),
+    ("loss_gqa_mapping", "const float* kj = k + (j * Hkv + hk) * (int64_t)dh;\n        double dot = 0.0;\n"
+     "        for (int32_t c = 0; c < dh; ++c) dot += (double)qi[c] * (double)kj[c];\n"
+     "        s[j - j0] = dot;",
+     "const float* kj = k + (j * Hkv + h % Hkv) * (int64_t)dh;\n        double dot = 0.0;\n"
+     "        for (int32_t c = 0; c < dh; ++c) dot += (double)qi[c] * (double)kj[c];\n"
+     "        s[j - j0] = dot;",
+     lambda o: pb.test_loss_is_the_forward_inner_product(o)),
 ]
 
 
