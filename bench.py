@@ -29,7 +29,9 @@ METRIC = "gated-prefill input tok/s"
 # the libtokengate kernel each stage launches on the tensor-core path (the attention
 # kernel depends on the batch: tg.attention_kernel names it)
 KERNELS = {"gate": "gate_tc2_kernel", "topk": "topk_kernel", "gather": "gather_bulk_kernel"}
+KERNELS_FP32 = {**KERNELS, "gate": "gate_simt_kernel"}  # fp32 gates run on the CUDA cores
 HOLD_CYCLES = 40_000_000  # ~20 ms of device time before each timed batch is queued
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # nominal FP32 FMA peak (CUDA-core fp32 path)
 
 
 def _peaks():
@@ -133,13 +135,160 @@ def _sha(path):
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
 
+DTYPES = {"bf16": "bf16", "fp32": "f32"}
+# every other configuration measured in the same process after the headline one:
+# (name, the workload whose inputs it reuses); the 32k budget sweep shares its inputs
+OTHER_WORKLOADS = [("tiny_fp32", "tiny_fp32"), ("qwen_32k_k1024", "qwen_32k_k1024"),
+                   ("qwen_32k_k4096", "qwen_32k_k1024"), ("qwen_32k_k8192", "qwen_32k_k1024"),
+                   ("qwen_128k", "qwen_128k"), ("ragged_4", "ragged_4")]
+
+
+def _make_layer(tg, inp, w, dev):
+    from learned_token_pruning_gate_b200.pipeline import GatedLayer
+
+    d = lambda t: t.to(dev).contiguous()  # noqa: E731
+    return GatedLayer(d(inp.h), d(inp.q), d(inp.k), d(inp.v), d(inp.W1), d(inp.b1), d(inp.w2),
+                      inp.b2, d(inp.gain), d(inp.temp), inp.cu_seqlens, inp.doc_begin,
+                      inp.doc_end, np.asarray(w.budgets, np.int32), rope_theta=w.rope_theta,
+                      algo=tg.ALGO_AUTO)
+
+
+def _time_steps(graph, flush, stream, K, warmup, settle_s=0.3):
+    """K CUDA-graph replays, each bracketed by CUDA events on the launching stream,
+    with an L2 flush between them (outside the events).  Returns per-step ms."""
+    import torch
+
+    t_warm = time.time()
+    for _ in range(max(warmup, 3)):
+        flush.zero_()
+        graph.replay()
+    while time.time() - t_warm < settle_s:  # let the clocks settle before timing
+        flush.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    # hold the stream for a moment so the host queues launches ahead of the GPU:
+    # the timed intervals then hold device work only, not host launch latency
+    torch.cuda._sleep(HOLD_CYCLES)
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        graph.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def _time_stages(layer, flush, stream, n):
+    """Each of the step's launches alone, n times, one event pair each (ms, mean)."""
+    import ctypes
+
+    import torch
+
+    kev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)] for s in layer.STAGES}
+    st = ctypes.c_void_p(stream.cuda_stream)
+    torch.cuda._sleep(HOLD_CYCLES)
+    for i in range(n):
+        flush.zero_()
+        for s in layer.STAGES:
+            kev[s][i][0].record(stream)
+            getattr(layer, s)(st)
+            kev[s][i][1].record(stream)
+    torch.cuda.synchronize()
+    return {s: float(np.mean([a.elapsed_time(b) for a, b in kev[s]])) for s in kev}
+
+
+def _stages_and_roofline(tg, layer, w, name, stage_ms, pk):
+    """Per-stage achieved rates and the roofline object of the dominant kernel."""
+    work = layer.work()
+    kernels = KERNELS if w.dtype == "bf16" else KERNELS_FP32
+    us = {s: stage_ms[s] * 1e3 for s in stage_ms}
+    stages = {
+        "gate": {"us": us["gate"], "tflops": work["gate_flops"] / us["gate"] / 1e6,
+                 "gbs": work["gate_bytes"] / us["gate"] / 1e3},
+        "topk": {"us": us["topk"], "gbs": work["topk_bytes"] / us["topk"] / 1e3},
+        "gather": {"us": us["gather"], "gbs": work["gather_bytes"] / us["gather"] / 1e3},
+        "attention": {"us": us["attention"],
+                      "tflops": work["attn_flops"] / us["attention"] / 1e6},
+    }
+    for s in stages.values():
+        if "tflops" in s:
+            s["frac_tensor"] = s["tflops"] / pk["bf16"]
+        if "gbs" in s:
+            s["frac_hbm"] = s["gbs"] / pk["hbm"]
+    tg_us = us["topk"] + us["gather"]
+    stages["topk+gather"] = {"us": tg_us,
+                             "gbs": (work["topk_bytes"] + work["gather_bytes"]) / tg_us / 1e3}
+    stages["topk+gather"]["frac_hbm"] = stages["topk+gather"]["gbs"] / pk["hbm"]
+    dominant = max(("gate", "topk", "gather", "attention"), key=lambda s: us[s])
+    attn_kernel = tg.attention_kernel(layer.cu_kept_host, w.n_q_heads, w.n_kv_heads, w.head_dim,
+                                      dtype=w.dtype, with_workspace=layer.workspace is not None)
+    attn_kernel = attn_kernel.split(" ")[0]
+    stages["attention"]["kernel"] = attn_kernel
+    if dominant == "attention" and w.dtype == "bf16":
+        roof = {"kernel": attn_kernel, "bound": "tensor",
+                "achieved": stages["attention"]["tflops"], "peak": pk["bf16"], "unit": "TFLOP/s"}
+    elif dominant == "attention":  # fp32 runs on the CUDA cores: FP32 FMA peak
+        roof = {"kernel": attn_kernel, "bound": "alu", "achieved": stages["attention"]["tflops"],
+                "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s"}
+    elif dominant == "gate":
+        t_flop = work["gate_flops"] / (pk["bf16"] * 1e12)
+        t_byte = work["gate_bytes"] / (pk["hbm"] * 1e9)
+        if t_flop >= t_byte:
+            roof = {"kernel": kernels["gate"], "bound": "tensor",
+                    "achieved": stages["gate"]["tflops"], "peak": pk["bf16"], "unit": "TFLOP/s"}
+        else:
+            roof = {"kernel": kernels["gate"], "bound": "hbm", "achieved": stages["gate"]["gbs"],
+                    "peak": pk["hbm"], "unit": "GB/s"}
+    else:
+        roof = {"kernel": kernels[dominant], "bound": "hbm",
+                "achieved": stages[dominant]["gbs"], "peak": pk["hbm"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = _traffic(roof["kernel"], name)
+    roof["peak_source"] = f"{pk['source']} (burst)" if roof["bound"] != "alu" else \
+        "nominal FP32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"
+    return stages, roof
+
+
+def _other_workloads(tg, gen, dev, stream, flush, pk, K):
+    """Every configuration besides the headline one, timed the same way (graph
+    replay, L2 flushed, CUDA events), fewer steps; buffers freed in between."""
+    import torch
+
+    res, cache = {}, {}
+    for name, src in OTHER_WORKLOADS:
+        w = gen.WORKLOADS[name]
+        if src not in cache:
+            cache.clear()
+            cache[src] = gen.make_inputs(gen.WORKLOADS[src])
+        inp = cache[src]
+        layer = _make_layer(tg, inp, w, dev)
+        graph = layer.capture()
+        with ClockSampler(dev.index or 0) as clocks:
+            step_ms = _time_steps(graph, flush, stream, K, 3, settle_s=0.1)
+        stage_ms = _time_stages(layer, flush, stream, min(K, 10))
+        if tg.device_status() != 0:
+            raise SystemExit(f"{name}: a kernel reported a timed-out wait")
+        stages, roof = _stages_and_roofline(tg, layer, w, name, stage_ms, pk)
+        ms = float(np.mean(step_ms))
+        res[name] = {"ms_per_step": ms, "tok_s": w.total_tokens / ms * 1e3, "steps": K,
+                     "dtype": DTYPES[w.dtype], "tokens": w.total_tokens,
+                     "kept_M": w.kept_lengths(), "stages": stages, "roofline": roof,
+                     "clocks": clocks.summary()}
+        del graph, layer
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_gpu(args):
     import torch
 
     import learned_token_pruning_gate_b200 as tg
     from learned_token_pruning_gate_b200 import inputs as gen
     from learned_token_pruning_gate_b200 import dist as tgd
-    from learned_token_pruning_gate_b200.pipeline import GatedLayer
 
     rank, world, local = _dist_init(args.gpus)
     torch.cuda.set_device(local)
@@ -147,59 +296,23 @@ def run_gpu(args):
     w = tgd.rank_workload(gen.WORKLOADS[args.workload], rank)
     inp = gen.make_inputs(w)
     dev = torch.device("cuda", local)
-    d = lambda t: t.to(dev).contiguous()  # noqa: E731
-    layer = GatedLayer(d(inp.h), d(inp.q), d(inp.k), d(inp.v), d(inp.W1), d(inp.b1), d(inp.w2),
-                       inp.b2, d(inp.gain), d(inp.temp), inp.cu_seqlens, inp.doc_begin,
-                       inp.doc_end, inp.budget, rope_theta=w.rope_theta, algo=tg.ALGO_AUTO)
+    layer = _make_layer(tg, inp, w, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     graph = layer.capture()
 
     # ---- device-timed steps (inputs resident in HBM), CUDA graph replay --------
-    t_warm = time.time()
-    for i in range(max(args.warmup, 3)):
-        flush.zero_()
-        graph.replay()
-    while time.time() - t_warm < 0.3:  # let the clocks settle before timing
-        flush.zero_()
-        graph.replay()
-        torch.cuda.synchronize()
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     tgd.barrier()
     with ClockSampler(local) as clocks:
-        # hold the stream for a moment so the host queues launches ahead of the GPU:
-        # the timed intervals then hold device work only, not host launch latency
-        torch.cuda._sleep(HOLD_CYCLES)
-        for i in range(K):
-            flush.zero_()  # L2 flush outside the timed interval
-            ev[i][0].record(stream)
-            graph.replay()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
+        step_ms = _time_steps(graph, flush, stream, K, args.warmup)
     tgd.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = tgd.max_over_ranks(float(np.sum(step_ms)), device=dev)
     if tg.device_status() != 0:
         raise SystemExit("a kernel reported a timed-out wait")
 
     # ---- per-kernel times for the roofline (same launches, one event pair each) --
-    n_k = min(K, 50)
-    kev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(n_k)] for s in GatedLayer.STAGES}
-    import ctypes
-
-    st = ctypes.c_void_p(stream.cuda_stream)
-    torch.cuda._sleep(HOLD_CYCLES)
-    for i in range(n_k):
-        flush.zero_()
-        for s in GatedLayer.STAGES:
-            kev[s][i][0].record(stream)
-            getattr(layer, s)(st)
-            kev[s][i][1].record(stream)
-    torch.cuda.synchronize()
-    stage_ms = {s: float(np.mean([a.elapsed_time(b) for a, b in kev[s]])) for s in kev}
+    stage_ms = _time_stages(layer, flush, stream, min(K, 50))
 
     # ---- end to end: pinned host inputs -> device -> 4 C-ABI calls -> host -----
     pinned = {n: getattr(inp, n).pin_memory() for n in ("h", "q", "k", "v")}
@@ -233,53 +346,14 @@ def run_gpu(args):
     # ---- report -------------------------------------------------------------------
     tokens = w.total_tokens
     value = tgd.aggregate_throughput(tokens, K, total_ms, world)
-    work = layer.work()
     pk = _peaks()
-    us = {s: stage_ms[s] * 1e3 for s in stage_ms}
-    stages = {
-        "gate": {"us": us["gate"], "tflops": work["gate_flops"] / us["gate"] / 1e6,
-                 "gbs": work["gate_bytes"] / us["gate"] / 1e3},
-        "topk": {"us": us["topk"], "gbs": work["topk_bytes"] / us["topk"] / 1e3},
-        "gather": {"us": us["gather"], "gbs": work["gather_bytes"] / us["gather"] / 1e3},
-        "attention": {"us": us["attention"],
-                      "tflops": work["attn_flops"] / us["attention"] / 1e6},
-    }
-    for s in stages.values():
-        if "tflops" in s:
-            s["frac_tensor"] = s["tflops"] / pk["bf16"]
-        if "gbs" in s:
-            s["frac_hbm"] = s["gbs"] / pk["hbm"]
-    tg_us = us["topk"] + us["gather"]
-    stages["topk+gather"] = {"us": tg_us,
-                             "gbs": (work["topk_bytes"] + work["gather_bytes"]) / tg_us / 1e3}
-    stages["topk+gather"]["frac_hbm"] = stages["topk+gather"]["gbs"] / pk["hbm"]
-    dominant = max(("gate", "topk", "gather", "attention"), key=lambda s: us[s])
-    attn_kernel = tg.attention_kernel(layer.cu_kept_host, w.n_q_heads, w.n_kv_heads, w.head_dim,
-                                      with_workspace=layer.workspace is not None).split(" ")[0]
-    if dominant == "attention":
-        roof = {"kernel": attn_kernel, "bound": "tensor",
-                "achieved": stages["attention"]["tflops"], "peak": pk["bf16"], "unit": "TFLOP/s"}
-    elif dominant == "gate":
-        t_flop = work["gate_flops"] / (pk["bf16"] * 1e12)
-        t_byte = work["gate_bytes"] / (pk["hbm"] * 1e9)
-        if t_flop >= t_byte:
-            roof = {"kernel": KERNELS["gate"], "bound": "tensor",
-                    "achieved": stages["gate"]["tflops"], "peak": pk["bf16"], "unit": "TFLOP/s"}
-        else:
-            roof = {"kernel": KERNELS["gate"], "bound": "hbm", "achieved": stages["gate"]["gbs"],
-                    "peak": pk["hbm"], "unit": "GB/s"}
-    else:
-        roof = {"kernel": KERNELS[dominant], "bound": "hbm",
-                "achieved": stages[dominant]["gbs"], "peak": pk["hbm"], "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = _traffic(roof["kernel"], args.workload)
-    roof["peak_source"] = f"{pk['source']} (burst)"
+    stages, roof = _stages_and_roofline(tg, layer, w, args.workload, stage_ms, pk)
     e2e_value = tgd.aggregate_throughput(tokens, n_e2e, e2e_ms, world)
 
     result = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": DTYPES[w.dtype], "data": "synthetic",
         "config": {**_workload_config(args.workload, w, world),
                    "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
                    "timing": "CUDA events per step around a CUDA-graph replay of the 4 launches"},
@@ -290,11 +364,18 @@ def run_gpu(args):
         "stages": stages,
         "clocks": clocks.summary(),
     }
+    del graph, layer, pinned
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(inp, seconds=args.cpu_seconds)
+    del inp
+    if world == 1 and not args.headline_only:
+        result["workloads"] = _other_workloads(tg, gen, dev, stream, flush, pk,
+                                               max(3, min(K, args.other_steps)))
+        result["gpu_launches_workloads"] = 4 * sum(
+            v["steps"] + 3 for v in result["workloads"].values())
     if rank == 0:
         print(json.dumps(result), flush=True)
-    del graph
     if world > 1:
         import torch.distributed as dist
 
@@ -633,6 +714,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other configurations' block (workloads)")
+    ap.add_argument("--other-steps", type=int, default=20,
+                    help="timed steps per configuration in the workloads block")
     ap.add_argument("--extras", action="store_true",
                     help="print bias overhead, ungated full-N attention and memory figures")
     ap.add_argument("--ncu-case", action="store_true",

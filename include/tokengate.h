@@ -100,6 +100,17 @@ TG_API const char* tg_version(void);
 TG_API tg_status tg_device_status(tg_stream_t stream, uint32_t* bits_out);
 
 /*
+ * The same read-and-clear of the device status word with the bits as a signed
+ * code (0 = no kernel reported a failure).  Synchronises `stream`; returns
+ * TG_ERR_DEVICE_CHECK when bits were set, TG_ERR_INVALID_ARG for a NULL
+ * code_out.  Bits: 1 a gate pipeline wait gave up, 2 an attention wait gave
+ * up (forward or backward), 4 the top-K selection produced more rows than M_b (extra rows skipped),
+ * 8 a kept index outside the prompt batch reached the gather (row skipped),
+ * 16 a gather pipeline wait gave up.
+ */
+TG_API tg_status tg_last_device_error(tg_stream_t stream, int32_t* code_out);
+
+/*
  * Host-only helper: validates a prompt batch and writes the kept-row offsets
  * cu_kept_h[0..batch] (cu_kept_h[b+1] - cu_kept_h[b] = M_b) so the caller can
  * size the outputs of the later calls.  All arrays are host memory.
@@ -279,9 +290,12 @@ TG_API tg_status tg_attention_kernel(tg_dtype dtype, int32_t batch, const int32_
  * library until the process exits.
  *   Arguments, results and errors are those of tg_gated_attention without the
  *   workspace.  A batch whose split plan needs more scratch than the array
- *   holds returns TG_ERR_WORKSPACE before anything launches.
+ *   holds runs the unsplit plan (each query tile on one SM), which needs none:
+ *   the results are the same up to rounding, only the schedule differs.
  *   The first call on a device looks up the array's address (a runtime call,
- *   no allocation): make it before any stream capture on that device.
+ *   no allocation): make it before any stream capture on that device.  The
+ *   address is looked up again when the device's context has changed (after a
+ *   cudaDeviceReset), so it never outlives the context it belongs to.
  *   All calls share the array: calls that run on the GPU at the same time race
  *   on it, so issue them in order on one stream.  The call allocates nothing.
  */

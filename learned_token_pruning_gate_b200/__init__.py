@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = (
     "tg_gated_attention", "tg_attention_workspace_bytes", "tg_attention_kernel",
     "tg_gated_attention_noalloc", "tg_topk_select_multi", "tg_random_select",
     "tg_gated_attention_backward", "tg_attention_backward_workspace_bytes", "tg_rmsnorm",
-    "tg_qkv_rope_emit", "tg_swiglu", "tg_gated_delta_scan",
+    "tg_qkv_rope_emit", "tg_swiglu", "tg_gated_delta_scan", "tg_last_device_error",
 )
 MAX_BUDGETS = 8
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
@@ -81,6 +81,7 @@ def library():
     L.tg_last_error_message.restype = ctypes.c_char_p
     L.tg_version.restype = ctypes.c_char_p
     L.tg_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.tg_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
     L.tg_kept_offsets.argtypes = [_i32, _i32p, _i32p, _i32p, _i32p, _i32p]
     L.tg_gate_score.argtypes = [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, _i32, _vp, _f32, _vp,
                                 _i32, _vp]
@@ -151,6 +152,22 @@ def _need_cuda(*ts):
             raise ValueError("libtokengate operates on CUDA tensors only")
 
 
+def _expect(name, t, shape, dtype, device):
+    """A caller-passed tensor must match what the call reads or writes exactly:
+    the kernels take raw pointers and trust the sizes derived from the other
+    arguments, so a smaller buffer would be read or written past its end."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
 def device_status(stream=None):
     """Synchronise and return (and clear) the device status bits (0 = no failure)."""
     bits = ctypes.c_uint32(0)
@@ -175,11 +192,16 @@ def kept_offsets(cu_seqlens, doc_begin, doc_end, budget) -> np.ndarray:
 
 def gate_score(h, W1, b1, w2, b2, out=None, algo=ALGO_AUTO):
     """z = w2 . GELU(W1 h + b1) + b2 for every row of h [n, d]."""
-    _need_cuda(h, W1, b1, w2)
     n, d = h.shape
     dg = W1.shape[0]
     if W1.shape[1] != d or W1.dtype != h.dtype:
         raise ValueError("W1 must be [d_hidden, d_model] with h's dtype")
+    _expect("h", h, (n, d), h.dtype, h.device)
+    _expect("W1", W1, (dg, d), h.dtype, h.device)
+    _expect("b1", b1, (dg,), torch.float32, h.device)
+    _expect("w2", w2, (dg,), torch.float32, h.device)
+    _expect("out", out, (n,), torch.float32, h.device)
+    _need_cuda(h, W1, b1, w2)
     if out is None:
         out = torch.empty(n, dtype=torch.float32, device=h.device)
     _check("tg_gate_score", library().tg_gate_score(
@@ -193,17 +215,22 @@ def topk_select(z, cu_seqlens, doc_begin, doc_end, budget, kept_idx=None, cu_kep
 
     Returns (kept_idx [M] int32 device, cu_kept [B+1] int32 device, cu_kept_host).
     """
-    _need_cuda(z)
     cu, cu_p = _host_i32(cu_seqlens)
     s, s_p = _host_i32(doc_begin)
     e, e_p = _host_i32(doc_end)
     k, k_p = _host_i32(budget)
     host = kept_offsets(cu, s, e, k)
     M = int(host[-1])
+    _expect("z", z, (int(cu[-1]),), torch.float32, z.device)
+    _expect("kept_idx", kept_idx, (M,), torch.int32, z.device)
+    _expect("cu_kept", cu_kept, (len(s) + 1,), torch.int32, z.device)
+    _need_cuda(z)
     if kept_idx is None:
         kept_idx = torch.empty(max(M, 1), dtype=torch.int32, device=z.device)[:M]
     if cu_kept is None:
         cu_kept = torch.empty(len(s) + 1, dtype=torch.int32, device=z.device)
+    _expect("kept_idx", kept_idx, (M,), torch.int32, z.device)
+    _expect("cu_kept", cu_kept, (len(s) + 1,), torch.int32, z.device)
     _check("tg_topk_select", library().tg_topk_select(
         _ptr(z), len(s), cu_p, s_p, e_p, k_p, _ptr(kept_idx), _ptr(cu_kept), _stream(z.device)))
     return kept_idx, cu_kept, host
@@ -219,6 +246,7 @@ def topk_select_multi(z, cu_seqlens, doc_begin, doc_end, budgets):
     cu, cu_p = _host_i32(cu_seqlens)
     s, s_p = _host_i32(doc_begin)
     e, e_p = _host_i32(doc_end)
+    _expect("z", z, (int(cu[-1]),), torch.float32, z.device)
     ks = np.ascontiguousarray(np.asarray(budgets, dtype=np.int32).reshape(len(budgets), len(s)))
     outs, kept_ptrs, cu_ptrs = [], (_vp * len(ks))(), (_vp * len(ks))()
     for q, k in enumerate(ks):
@@ -245,6 +273,7 @@ def random_select(keys, cu_seqlens, doc_begin, doc_end, budget):
     k, k_p = _host_i32(budget)
     host = kept_offsets(cu, s, e, k)
     M = int(host[-1])
+    _expect("keys", keys, (int(cu[-1]),), torch.int32, keys.device)
     kept_idx = torch.empty(max(M, 1), dtype=torch.int32, device=keys.device)[:M]
     cu_kept = torch.empty(len(s) + 1, dtype=torch.int32, device=keys.device)
     _check("tg_random_select", library().tg_random_select(
@@ -261,7 +290,6 @@ def compact_gather(kept_idx, cu_seqlens, doc_begin, doc_end, budget, tensors, ro
     """
     if len(tensors) > MAX_GATHER_TENSORS:
         raise ValueError("too many tensors")
-    _need_cuda(kept_idx, z, *tensors)
     cu, cu_p = _host_i32(cu_seqlens)
     s, s_p = _host_i32(doc_begin)
     e, e_p = _host_i32(doc_end)
@@ -272,9 +300,23 @@ def compact_gather(kept_idx, cu_seqlens, doc_begin, doc_end, budget, tensors, ro
         raise ValueError("all gathered tensors must share one dtype")
     dcode = _dtype_code(tensors[0]) if tensors else TG_BF16
     rope_heads = rope_heads or [0] * len(tensors)
+    dev0 = tensors[0].device if tensors else kept_idx.device
+    _expect("kept_idx", kept_idx, (M,), torch.int32, dev0)
+    N = int(cu[-1])
+    for i, t in enumerate(tensors):
+        _expect(f"tensors[{i}]", t, (N,) + tuple(t.shape[1:]), tensors[0].dtype, dev0)
+    if z is not None:
+        _expect("z", z, (N,), torch.float32, dev0)
     if outs is None:
         outs = [torch.empty((M,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
                 for t in tensors]
+    if len(outs) != len(tensors):
+        raise ValueError("one output per gathered tensor")
+    for i, (t, o) in enumerate(zip(tensors, outs)):
+        _expect(f"outs[{i}]", o, (M,) + tuple(t.shape[1:]), t.dtype, dev0)
+    if logsig_out is not None:
+        _expect("logsig_out", logsig_out, (M,), torch.float32, dev0)
+    _need_cuda(kept_idx, z, *tensors)
     arr = (GatherTensor * max(len(tensors), 1))()
     for i, (src, dst) in enumerate(zip(tensors, outs)):
         if not src.is_contiguous() or not dst.is_contiguous():
@@ -290,6 +332,24 @@ def compact_gather(kept_idx, cu_seqlens, doc_begin, doc_end, budget, tensors, ro
         _ptr(kept_idx), M, len(s), cu_p, s_p, e_p, k_p, dcode, arr, len(tensors), head_dim,
         float(rope_theta), _ptr(z), _ptr(logsig_out), _stream(dev)))
     return outs, logsig_out
+
+
+def _attention_operands(q, k, v, logsig, gain, temp):
+    """q [M, Hq, d], k and v [M, Hkv, d] of one dtype on one device, contiguous;
+    logsig [M], gain and temp [Hq] fp32.  The kernels read k and v with q's
+    element size and row count, so any mismatch would read past their end."""
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k and v must be [rows, heads, head_dim]")
+    M, Hq, dh = q.shape
+    Hkv = k.shape[1]
+    if Hkv <= 0 or Hq % Hkv != 0:
+        raise ValueError(f"{Hq} query heads are not a multiple of {Hkv} kv heads")
+    _expect("q", q, (M, Hq, dh), q.dtype, q.device)
+    _expect("k", k, (M, Hkv, dh), q.dtype, q.device)
+    _expect("v", v, (M, Hkv, dh), q.dtype, q.device)
+    _expect("logsig", logsig, (M,), torch.float32, q.device)
+    _expect("gain", gain, (Hq,), torch.float32, q.device)
+    _expect("temp", temp, (Hq,), torch.float32, q.device)
 
 
 def attention_workspace_bytes(cu_kept_host, n_q_heads, n_kv_heads, head_dim, dtype="bf16",
@@ -323,10 +383,19 @@ def gated_attention(q, k, v, cu_kept_host, logsig=None, gain=None, temp=None, ou
     workspace: "auto" (allocate what the call can use), None (no split), or a
     uint8 device tensor.  Returns (out [M, Hq, d], lse [Hq, M] or None).
     """
-    _need_cuda(q, k, v, logsig, gain, temp)
+    _attention_operands(q, k, v, logsig, gain, temp)
     M, Hq, dh = q.shape
     Hkv = k.shape[1]
     cu, cu_p = _host_i32(cu_kept_host)
+    if int(cu[-1]) != M:
+        raise ValueError(f"cu_kept_host ends at {int(cu[-1])}, q has {M} rows")
+    _expect("out", out, (M, Hq, dh), q.dtype, q.device)
+    _expect("lse", lse, (Hq, M), torch.float32, q.device)
+    if workspace is not None and not isinstance(workspace, str):
+        if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or \
+                workspace.device != q.device:
+            raise ValueError("workspace must be a contiguous uint8 tensor on q's device")
+    _need_cuda(q, k, v, logsig, gain, temp)
     if out is None:
         out = torch.empty_like(q)
     if want_lse and lse is None:
@@ -359,10 +428,21 @@ def gated_attention_backward(q, k, v, cu_kept_host, logsig, gain, temp, out, lse
     dout = dL/dout [M, Hq, d]; out, lse = the forward's outputs (lse [Hq, M]).
     Returns (d_logsig [M], d_z_kept [M], d_gain [Hq], d_temp [Hq]), fp32 device.
     """
-    _need_cuda(q, k, v, logsig, gain, temp, out, lse, dout)
+    _attention_operands(q, k, v, logsig, gain, temp)
     M, Hq, dh = q.shape
     Hkv = k.shape[1]
+    if logsig is None or lse is None:
+        raise ValueError("the backward needs the log-gates and the forward's lse")
+    _expect("out", out, (M, Hq, dh), q.dtype, q.device)
+    _expect("dout", dout, (M, Hq, dh), q.dtype, q.device)
+    _expect("lse", lse, (Hq, M), torch.float32, q.device)
     cu, cu_p = _host_i32(cu_kept_host)
+    if int(cu[-1]) != M:
+        raise ValueError(f"cu_kept_host ends at {int(cu[-1])}, q has {M} rows")
+    if workspace is not None and (workspace.dtype != torch.uint8 or
+                                  not workspace.is_contiguous() or workspace.device != q.device):
+        raise ValueError("workspace must be a contiguous uint8 tensor on q's device")
+    _need_cuda(q, k, v, logsig, gain, temp, out, lse, dout)
     if workspace is None:
         workspace = torch.empty(attention_backward_workspace_bytes(cu, Hq), dtype=torch.uint8,
                                 device=q.device)
@@ -378,8 +458,11 @@ def gated_attention_backward(q, k, v, cu_kept_host, logsig, gain, temp, out, lse
 
 def rmsnorm(x, weight, eps=1e-6, out=None):
     """x / sqrt(mean(x^2) + eps) * weight over the last axis of x [rows, dim]."""
-    _need_cuda(x, weight)
     rows, dim = x.shape
+    _expect("x", x, (rows, dim), x.dtype, x.device)
+    _expect("weight", weight, (dim,), x.dtype, x.device)
+    _expect("out", out, (rows, dim), x.dtype, x.device)
+    _need_cuda(x, weight)
     if out is None:
         out = torch.empty_like(x)
     _check("tg_rmsnorm", library().tg_rmsnorm(_ptr(x), _ptr(weight), _ptr(out), _dtype_code(x),
@@ -392,10 +475,19 @@ def qkv_rope_emit(qkv, cu_seqlens, cu_kept_host, kept_idx, n_q_heads, n_kv_heads
                   v_out=None):
     """Split a fused QKV projection [M, (Hq + 2 Hkv) d] into q (per-head RMSNorm,
     RoPE), k (same; the layer's KV-cache slot) and v.  Returns (q, k, v)."""
-    _need_cuda(qkv, kept_idx, q_norm_w, k_norm_w)
     M = qkv.shape[0]
     cu, cu_p = _host_i32(cu_seqlens)
     ck, ck_p = _host_i32(cu_kept_host)
+    if int(ck[-1]) != M:
+        raise ValueError(f"cu_kept_host ends at {int(ck[-1])}, qkv has {M} rows")
+    _expect("qkv", qkv, (M, (n_q_heads + 2 * n_kv_heads) * head_dim), qkv.dtype, qkv.device)
+    _expect("kept_idx", kept_idx, (M,), torch.int32, qkv.device)
+    _expect("q_norm_w", q_norm_w, (head_dim,), qkv.dtype, qkv.device)
+    _expect("k_norm_w", k_norm_w, (head_dim,), qkv.dtype, qkv.device)
+    _expect("q_out", q_out, (M, n_q_heads, head_dim), qkv.dtype, qkv.device)
+    _expect("k_out", k_out, (M, n_kv_heads, head_dim), qkv.dtype, qkv.device)
+    _expect("v_out", v_out, (M, n_kv_heads, head_dim), qkv.dtype, qkv.device)
+    _need_cuda(qkv, kept_idx, q_norm_w, k_norm_w)
     mk = lambda h: torch.empty((M, h, head_dim), dtype=qkv.dtype, device=qkv.device)  # noqa: E731
     q_out = mk(n_q_heads) if q_out is None else q_out
     k_out = mk(n_kv_heads) if k_out is None else k_out
@@ -409,8 +501,12 @@ def qkv_rope_emit(qkv, cu_seqlens, cu_kept_host, kept_idx, n_q_heads, n_kv_heads
 
 def swiglu(gate_up, out=None):
     """SiLU(gate) * up of a fused [rows, 2 inter] projection."""
-    _need_cuda(gate_up)
     rows, two = gate_up.shape
+    if two % 2:
+        raise ValueError("gate_up must hold the gate and up halves side by side")
+    _expect("gate_up", gate_up, (rows, two), gate_up.dtype, gate_up.device)
+    _expect("out", out, (rows, two // 2), gate_up.dtype, gate_up.device)
+    _need_cuda(gate_up)
     if out is None:
         out = torch.empty((rows, two // 2), dtype=gate_up.dtype, device=gate_up.device)
     _check("tg_swiglu", library().tg_swiglu(_ptr(gate_up), _ptr(out), _dtype_code(gate_up), rows,
@@ -431,14 +527,17 @@ def gated_delta_scan(q, k, v, cu_kept_host, log_alpha, beta, eps=1e-6, out=None,
         raise ValueError(f"log_alpha and beta must be [M, H] = {(M, H)}")
     if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
         raise ValueError("log_alpha and beta must be float32")
-    for t in (q, k, v, log_alpha, beta):
-        if not t.is_contiguous():
-            raise ValueError("gated_delta_scan takes contiguous tensors")
-    _need_cuda(q, k, v, log_alpha, beta)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _expect(name, t, (M, H, d), q.dtype, q.device)
+    _expect("log_alpha", log_alpha, (M, H), torch.float32, q.device)
+    _expect("beta", beta, (M, H), torch.float32, q.device)
     ck, ck_p = _host_i32(cu_kept_host)
     if int(ck[-1]) != M:
         raise ValueError(f"cu_kept_host ends at {int(ck[-1])}, q has {M} rows")
     B = len(ck) - 1
+    _expect("out", out, (M, H, d), q.dtype, q.device)
+    _expect("state", state, (B, H, d, d), torch.float32, q.device)
+    _need_cuda(q, k, v, log_alpha, beta)
     if out is None:
         out = torch.empty_like(v)
     if state is None and want_state:

@@ -26,22 +26,58 @@ tg_status cuda_check(cudaError_t e, const char* what) {
   return set_error(TG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// Unique id of the calling thread's current CUDA context (0 when unavailable).
+// Device addresses of the library's __device__ arrays belong to one context: a
+// cudaDeviceReset destroys the primary context, and the next call runs in a new
+// one with the module loaded again, possibly elsewhere.  Context ids are never
+// reused within a process, so a cache keyed on them cannot hand out an address
+// of a destroyed context.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+uint64_t current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(id) + 1;  // 0 stays "unknown"
+}
+
+void* SymbolAddressCache::get(const void* symbol) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu_);
+  const uint64_t ctx = current_context_id();
+  if (addr_[dev] && ctx != 0 && ctx == ctx_[dev]) return addr_[dev];
+  // the lookup makes the device's primary context current when none is yet
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+  addr_[dev] = p;
+  ctx_[dev] = current_context_id();  // 0 (unknown) makes every call look the address up
+  return p;
+}
+
 // The status word lives in device global memory of each GPU that loaded the
 // library; kernels only ever atomically OR bits into it.
 static __device__ uint32_t g_status_word;
 
 uint32_t* device_status_word() {
-  static std::mutex mu;
-  static uint32_t* addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<uint32_t*>(p);
-  }
-  return addr[dev];
+  static SymbolAddressCache cache;
+  return static_cast<uint32_t*>(cache.get(reinterpret_cast<const void*>(&g_status_word)));
 }
 
 int num_sms() {
@@ -193,6 +229,14 @@ tg_status tg_device_status(tg_stream_t stream, uint32_t* bits_out) {
     return set_error(TG_ERR_DEVICE_CHECK, "device status bits 0x%x", bits);
   }
   return TG_OK;
+}
+
+tg_status tg_last_device_error(tg_stream_t stream, int32_t* code_out) {
+  if (!code_out) return set_error(TG_ERR_INVALID_ARG, "code_out is null");
+  uint32_t bits = 0;
+  const tg_status r = tg_device_status(stream, &bits);
+  *code_out = static_cast<int32_t>(bits);
+  return r;
 }
 
 tg_status tg_kept_offsets(int32_t batch, const int32_t* cu, const int32_t* s, const int32_t* e,

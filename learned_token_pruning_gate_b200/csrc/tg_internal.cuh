@@ -9,6 +9,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/tokengate.h"
 
 namespace tg {
@@ -38,6 +40,22 @@ enum : uint32_t {
 tg_status set_error(tg_status s, const char* fmt, ...);
 tg_status cuda_check(cudaError_t e, const char* what);
 uint32_t* device_status_word();  // device address for the current device (nullptr on failure)
+uint64_t current_context_id();    // unique id of the current CUDA context, 0 if unknown
+
+// Per-device cache of a __device__ symbol's address, looked up with
+// cudaGetSymbolAddress (a runtime call that allocates nothing) the first time
+// a device asks and again whenever that device's current context has changed
+// (after a cudaDeviceReset the module lives in a new context).
+class SymbolAddressCache {
+ public:
+  void* get(const void* symbol);
+
+ private:
+  static constexpr int kDevices = 64;
+  std::mutex mu_;
+  void* addr_[kDevices] = {};
+  uint64_t ctx_[kDevices] = {};
+};
 int num_sms();
 
 // Kernel launchers (each validates nothing: the C ABI layer has done it).

@@ -11,15 +11,17 @@
 //
 // The array lives in device memory of every GPU whose context loads the
 // library, until the process exits (kScratchBytes per GPU).  Its device address
-// is looked up once per device, on that device's first call (make the first
-// call before any stream capture).  All calls share the array, so two calls
-// that run on the GPU at the same time -- on different streams, or from
-// different threads -- race on it; order them on one stream.  Each call clears
-// the array's arrival counters on its stream before the kernel runs (the
-// attention launch does this for any workspace), nothing else must start at
-// zero.
-#include <mutex>
-
+// is looked up with cudaGetSymbolAddress (a runtime call that allocates
+// nothing) on a device's first call, and again when that device's current
+// context has changed -- after a cudaDeviceReset the module is loaded anew in a
+// new context, so an address kept from before would point at freed memory.
+// Make the first call on a device before any stream capture.  A batch whose
+// split plan needs more than the array holds runs the unsplit plan instead,
+// which needs no scratch.  All calls share the array, so two calls that run on
+// the GPU at the same time -- on different streams, or from different threads
+// -- race on it; order them on one stream.  Each call clears the array's
+// arrival counters on its stream before the kernel runs (the attention launch
+// does this for any workspace); nothing else must start at zero.
 #include "tg_internal.cuh"
 
 namespace tg {
@@ -29,19 +31,10 @@ constexpr size_t kScratchBytes = size_t(32) << 20;  // 32 MiB
 
 static __device__ __align__(256) uint8_t g_attn_scratch[kScratchBytes];
 
-// Device address of the array for the current device (nullptr on failure).
+// Device address of the array in the current context (nullptr on failure).
 void* scratch_address() {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  static SymbolAddressCache cache;
+  return cache.get(reinterpret_cast<const void*>(&g_attn_scratch));
 }
 
 }  // namespace
@@ -60,11 +53,9 @@ tg_status tg_gated_attention_noalloc(const void* q, const void* k, const void* v
   tg_status r = tg_attention_workspace_bytes(dtype, batch, cu_kept_h, n_q_heads, n_kv_heads,
                                              head_dim, algo, &need);
   if (r != TG_OK) return r;
-  if (need > kScratchBytes)
-    return set_error(TG_ERR_WORKSPACE,
-                     "this batch needs %zu bytes of attention scratch; the built-in array of "
-                     "tg_gated_attention_noalloc holds %zu (use tg_gated_attention with a workspace)",
-                     need, kScratchBytes);
+  if (need == 0 || need > kScratchBytes)  // no split, or a split the array cannot hold
+    return tg_gated_attention(q, k, v, dtype, batch, cu_kept_h, n_q_heads, n_kv_heads, head_dim,
+                              logsig, gain, temp, out, lse, nullptr, 0, algo, stream);
   void* scratch = scratch_address();
   if (!scratch) return set_error(TG_ERR_CUDA, "cannot resolve the attention scratch array");
   return tg_gated_attention(q, k, v, dtype, batch, cu_kept_h, n_q_heads, n_kv_heads, head_dim,

@@ -116,6 +116,34 @@ def _normal(rng, shape, std=1.0):
     return rng.standard_normal(size=shape, dtype=np.float32) * np.float32(std)
 
 
+_CHUNK_ROWS = 4096
+
+
+def _normal_rows(seed, stream, shape, dtype):
+    """N(0, 1) rows of a large tensor, drawn in chunks of _CHUNK_ROWS rows, chunk c
+    from its own Philox stream keyed by (seed, stream, c): the values depend only
+    on the seed, and the chunks are drawn on several threads (numpy releases the
+    GIL while it fills an array).  Returned as a torch tensor of ``dtype``."""
+    import concurrent.futures as cf
+    import os
+
+    n = shape[0]
+    row = int(np.prod(shape[1:])) if len(shape) > 1 else 1
+    out = torch.empty(shape, dtype=dtype)
+    flat = out.view(n, row)
+
+    def chunk(c):
+        lo, hi = c * _CHUNK_ROWS, min(n, (c + 1) * _CHUNK_ROWS)
+        g = np.random.Generator(np.random.Philox(key=[seed, (stream << 32) | c]))
+        block = g.standard_normal(size=(hi - lo, row), dtype=np.float32)
+        flat[lo:hi] = torch.from_numpy(block).to(dtype)
+
+    n_chunks = (n + _CHUNK_ROWS - 1) // _CHUNK_ROWS
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(chunk, range(n_chunks)))
+    return out
+
+
 def make_inputs(w: Workload, with_qkv: bool = True) -> Inputs:
     """Draw every input of workload ``w`` from its seed (numpy Philox)."""
     rng = np.random.Generator(np.random.Philox(w.seed))
@@ -132,29 +160,30 @@ def make_inputs(w: Workload, with_qkv: bool = True) -> Inputs:
     w2 = torch.from_numpy(_normal(rng, (w.d_hidden,), 0.02))
     b2 = float(_normal(rng, (1,), 0.02)[0])
 
-    h32 = _normal(rng, (w.total_tokens, w.d_model))
+    # the residual rows in fp32 first: the needle is added before the rounding
+    h32 = _normal_rows(w.seed, 1, (w.total_tokens, w.d_model), torch.float32)
     # Needle direction: W1^T w2 (the residual direction that raises the hidden
     # units with positive output weight and lowers the others), unit length.
     W1f = W1.float().numpy()
     direction = W1f.T.astype(np.float64) @ w2.numpy().astype(np.float64)
     direction /= np.linalg.norm(direction)
-    push = (NEEDLE_BETA * np.sqrt(w.d_model) * direction).astype(np.float32)
+    push = torch.from_numpy((NEEDLE_BETA * np.sqrt(w.d_model) * direction).astype(np.float32))
     needle_rows = []
     for b in range(B):
         n_doc = int(doc_end[b] - doc_begin[b])
         ln = min(w.needle, n_doc)
         off = int(rng.integers(0, max(n_doc - ln, 0) + 1))
         rows = np.arange(cu[b] + doc_begin[b] + off, cu[b] + doc_begin[b] + off + ln)
-        h32[rows] += push
+        h32[torch.from_numpy(rows)] += push
         needle_rows.append(rows.astype(np.int64))
-    h = torch.from_numpy(h32).to(dt)
+    h = h32.to(dt)
     del h32
 
     N = w.total_tokens
     if with_qkv:
-        q = torch.from_numpy(_normal(rng, (N, w.n_q_heads, w.head_dim))).to(dt)
-        k = torch.from_numpy(_normal(rng, (N, w.n_kv_heads, w.head_dim))).to(dt)
-        v = torch.from_numpy(_normal(rng, (N, w.n_kv_heads, w.head_dim))).to(dt)
+        q = _normal_rows(w.seed, 2, (N, w.n_q_heads, w.head_dim), dt)
+        k = _normal_rows(w.seed, 3, (N, w.n_kv_heads, w.head_dim), dt)
+        v = _normal_rows(w.seed, 4, (N, w.n_kv_heads, w.head_dim), dt)
     else:
         q = k = v = None
     gain = torch.from_numpy(rng.uniform(0.0, 1.0, w.n_q_heads).astype(np.float32))

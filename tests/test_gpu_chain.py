@@ -6,8 +6,8 @@ import torch
 
 import learned_token_pruning_gate_b200 as tg
 from learned_token_pruning_gate_b200 import inputs as gen
-from tests.parity_utils import (ATTN_BF16, ATTN_FP32, GATE_ATOL, assert_close, dev, host_f32,
-                                kept_set_agrees, sample_rows)
+from tests.parity_utils import (ATTN_BF16, ATTN_FP32, GATE_ATOL, LSE_ATOL, assert_close, dev,
+                                host_f32, kept_set_agrees, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,20 +30,65 @@ def _run_gpu(inp, algo=tg.ALGO_AUTO):
 
 
 def _oracle_chain(oracle, inp, rows=None):
+    """The oracle's own chain from the raw inputs (its scores, its selection)."""
     w = inp.w
     z = oracle.gate_score(inp.f32("h"), inp.f32("W1"), inp.b1.numpy(), inp.w2.numpy(), inp.b2)
     z32 = z.astype(np.float32)
     kept, cu_kept = oracle.topk_select(z32, inp.cu_seqlens, inp.doc_begin, inp.doc_end,
                                        inp.budget)
+    return dict(z=z, kept=kept, cu_kept=cu_kept)
+
+
+def _oracle_tail(oracle, inp, kept, cu_kept, z32, rows):
+    """Compaction and attention of the oracle on a given kept set and given scores
+    (the GPU's): always well defined, so the attention is always compared."""
+    w = inp.w
     q = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("q"), w.n_q_heads, w.head_dim,
                            w.rope_theta)
     k = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("k"), w.n_kv_heads, w.head_dim,
                            w.rope_theta)
     v = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("v"))
     ls = oracle.logsig(kept, inp.cu_seqlens, inp.doc_begin, inp.doc_end, z32)
-    out, lse = oracle.gated_attention(q, k, v, cu_kept, ls, inp.gain.numpy(), inp.temp.numpy(),
-                                      rows=rows)
-    return dict(z=z, kept=kept, cu_kept=cu_kept, out=out, lse=lse)
+    return oracle.gated_attention(q, k, v, cu_kept, ls, inp.gain.numpy(), inp.temp.numpy(),
+                                  rows=rows)
+
+
+def _check_chain(oracle, inp, g, rows=None, gate_rows=None):
+    """Every stage of the GPU chain against the oracle:
+      - gate scores within 1e-3 (all rows, or the sampled gate_rows);
+      - the selection bit-exact against the oracle's top-K on the GPU's scores,
+        and, when the oracle scored every row, within the 1e-3 band of its own;
+      - the planted needle kept;
+      - the attention output (and LSE) against the oracle's compaction and
+        attention over the GPU's kept set and scores, at the dtype's bar."""
+    w = inp.w
+    z = g["z"].cpu().numpy()
+    kept = g["kept_idx"].cpu().numpy()
+    cu_kept = g["cu_kept"].cpu().numpy()
+    if gate_rows is None:
+        ref = _oracle_chain(oracle, inp)
+        assert_close("z", z, ref["z"], GATE_ATOL, 0.0)
+        ok, ndiff = kept_set_agrees(kept, ref["kept"], ref["z"], inp.cu_seqlens, inp.doc_begin,
+                                    inp.doc_end, inp.budget)
+        assert ok, f"kept sets differ beyond the 1e-3 band ({ndiff} tokens)"
+    else:
+        zr = oracle.gate_score(inp.f32("h"), inp.f32("W1"), inp.b1.numpy(), inp.w2.numpy(),
+                               inp.b2, rows=gate_rows)
+        assert_close("z", z[gate_rows], zr, GATE_ATOL, 0.0)
+    ref_kept, ref_cu = oracle.topk_select(z, inp.cu_seqlens, inp.doc_begin, inp.doc_end,
+                                          inp.budget)
+    np.testing.assert_array_equal(kept, ref_kept)
+    np.testing.assert_array_equal(cu_kept, ref_cu)
+    for rows_b in inp.needle_rows:  # the planted needle always survives
+        assert set(rows_b.tolist()) <= set(kept.tolist())
+    out_ref, lse_ref = _oracle_tail(oracle, inp, kept, cu_kept, z, rows)
+    got = host_f32(g["out"])
+    lse = g["lse"].cpu().numpy().T  # [M, Hq]
+    if rows is not None:
+        got, lse = got[rows], lse[rows]
+    tol = ATTN_FP32 if w.dtype == "fp32" else ATTN_BF16
+    assert_close("out", got, out_ref, *tol)
+    assert_close("lse", lse, lse_ref, LSE_ATOL, 0.0)
 
 
 @pytest.mark.parametrize("name,algo", [("tiny_fp32", tg.ALGO_AUTO), ("tiny_fp32", tg.ALGO_SIMT),
@@ -54,27 +99,15 @@ def test_chain_matches_oracle(oracle, name, algo):
     g = _run_gpu(inp, algo)
     M = int(g["cu_kept_host"][-1])
     rows = None if w.total_tokens <= 4096 else sample_rows(M, g["cu_kept_host"], 24, seed=1)
-    ref = _oracle_chain(oracle, inp, rows)
-    assert_close("z", g["z"].cpu().numpy(), ref["z"], GATE_ATOL, 0.0)
-    ok, ndiff = kept_set_agrees(g["kept_idx"].cpu().numpy(), ref["kept"], ref["z"], inp.cu_seqlens,
-                                inp.doc_begin, inp.doc_end, inp.budget)
-    assert ok, f"kept sets differ beyond the 1e-3 band ({ndiff} tokens)"
-    for rows_b in inp.needle_rows:  # the planted needle always survives
-        assert set(rows_b.tolist()) <= set(g["kept_idx"].cpu().numpy().tolist())
-    if ndiff == 0:
-        got = host_f32(g["out"])
-        if rows is not None:
-            got = got[rows]
-        tol = ATTN_FP32 if w.dtype == "fp32" else ATTN_BF16
-        # bf16 chain: the oracle attends over fp64 RoPE'd q/k while the GPU stores them
-        # in bf16 first, so the bf16 bar applies; fp32 chain: the fp32 bar.
-        assert_close("out", got, ref["out"], *tol)
+    _check_chain(oracle, inp, g, rows)
 
 
-@pytest.mark.parametrize("name", ["qwen_128k", "ragged_4"])
-def test_chain_full_size_properties(oracle, name):
-    """Full-size chain: sampled gate scores against the oracle, and the selection
-    properties checked on the GPU's own scores (top-K is exact for given scores)."""
+@pytest.mark.parametrize("name", ["qwen_32k_k1024", "qwen_32k_k4096", "qwen_32k_k8192",
+                                  "qwen_128k", "ragged_4"])
+def test_chain_full_size_sampled(oracle, name):
+    """Full-size chain on sampled rows: gate scores on sampled tokens, the
+    selection bit-exact on the GPU's scores plus its properties, and the
+    attention of sampled query rows over the GPU's kept set."""
     w = gen.WORKLOADS[name]
     inp = gen.make_inputs(w)
     g = _run_gpu(inp)
@@ -83,10 +116,11 @@ def test_chain_full_size_properties(oracle, name):
     cu_kept = g["cu_kept"].cpu().numpy()
     np.testing.assert_array_equal(cu_kept, np.concatenate([[0], np.cumsum(w.kept_lengths())]))
     rng = np.random.default_rng(0)
-    rows = rng.integers(0, w.total_tokens, 256)
-    ref = oracle.gate_score(inp.f32("h"), inp.f32("W1"), inp.b1.numpy(), inp.w2.numpy(), inp.b2,
-                            rows=rows)
-    assert_close("z", z[rows], ref, GATE_ATOL, 0.0)
+    gate_rows = np.unique(np.concatenate([rng.integers(0, w.total_tokens, 256),
+                                          np.concatenate(inp.needle_rows)[:64]]))
+    M = int(cu_kept[-1])
+    rows = sample_rows(M, cu_kept, 24, seed=M)
+    _check_chain(oracle, inp, g, rows, gate_rows)
     for b in range(w.batch):
         s = inp.cu_seqlens[b] + inp.doc_begin[b]
         e = inp.cu_seqlens[b] + inp.doc_end[b]
@@ -99,7 +133,6 @@ def test_chain_full_size_properties(oracle, name):
             assert z[doc_kept].min() >= z[dropped].max()
         assert set(range(inp.cu_seqlens[b + 1] - w.question[b], inp.cu_seqlens[b + 1])) <= set(
             kb.tolist())
-        assert set(inp.needle_rows[b].tolist()) <= set(kb.tolist())
     assert np.isfinite(host_f32(g["out"])).all()
 
 
@@ -108,14 +141,7 @@ def test_chain_edge_cases(oracle):
     w = gen.Workload("edges", (0, 1, 300, 257, 64, 130), (0, 1, 300, 7, 0, 2),
                      (5, 1, 10, 0, 1000, 64), 128, 32, 4, 2, 64, "bf16", 2, 21)
     inp = gen.make_inputs(w)
-    g = _run_gpu(inp)
-    ref = _oracle_chain(oracle, inp)
-    assert_close("z", g["z"].cpu().numpy(), ref["z"], GATE_ATOL, 0.0)
-    ok, ndiff = kept_set_agrees(g["kept_idx"].cpu().numpy(), ref["kept"], ref["z"], inp.cu_seqlens,
-                                inp.doc_begin, inp.doc_end, inp.budget)
-    assert ok
-    if ndiff == 0:
-        assert_close("out", host_f32(g["out"]), ref["out"], *ATTN_BF16)
+    _check_chain(oracle, inp, _run_gpu(inp))
 
 
 def test_chain_maximum_batch(oracle):
@@ -129,11 +155,4 @@ def test_chain_maximum_batch(oracle):
     w = gen.Workload("max_batch", tuple(int(x) for x in seq), tuple(int(x) for x in qn),
                      tuple(int(x) for x in bud), 128, 32, 4, 2, 64, "bf16", 0, 92)
     inp = gen.make_inputs(w)
-    g = _run_gpu(inp)
-    ref = _oracle_chain(oracle, inp)
-    assert_close("z", g["z"].cpu().numpy(), ref["z"], GATE_ATOL, 0.0)
-    ok, ndiff = kept_set_agrees(g["kept_idx"].cpu().numpy(), ref["kept"], ref["z"], inp.cu_seqlens,
-                                inp.doc_begin, inp.doc_end, inp.budget)
-    assert ok
-    if ndiff == 0:
-        assert_close("out", host_f32(g["out"]), ref["out"], *ATTN_BF16)
+    _check_chain(oracle, inp, _run_gpu(inp))

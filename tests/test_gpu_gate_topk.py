@@ -54,7 +54,8 @@ def test_gate_parity(oracle, n, d, dg, dtype, algo):
         assert_close("z(fp32)", z.cpu().numpy(), ref, 2e-5, 0.0)
 
 
-@pytest.mark.parametrize("name", ["qwen_16k", "qwen_128k", "ragged_4"])
+@pytest.mark.parametrize("name", ["qwen_16k", "qwen_32k_k1024", "qwen_32k_k4096",
+                                  "qwen_32k_k8192", "qwen_128k", "ragged_4"])
 def test_gate_full_size_sampled(oracle, name):
     w = gen.WORKLOADS[name]
     inp = gen.make_inputs(w, with_qkv=False)

@@ -51,7 +51,8 @@ def _gather_case(oracle, w, seed):
     assert_close("logsig", ls.cpu().numpy(), ref_ls, *LOGSIG_TOL)
 
 
-@pytest.mark.parametrize("name", ["tiny_fp32", "qwen_16k", "qwen_128k", "ragged_4"])
+@pytest.mark.parametrize("name", ["tiny_fp32", "qwen_16k", "qwen_32k_k1024", "qwen_32k_k4096",
+                                  "qwen_32k_k8192", "qwen_128k", "ragged_4"])
 def test_gather_parity(oracle, name):
     _gather_case(oracle, gen.WORKLOADS[name], seed=11)
 
@@ -142,7 +143,8 @@ def test_attention_gain_zero_temp_one_is_plain_causal(oracle):
     assert_close("sdpa", host_f32(out), ref.cpu().numpy(), *ATTN_BF16)
 
 
-@pytest.mark.parametrize("name", ["qwen_16k", "qwen_128k", "ragged_4", "qwen_32k_k8192"])
+@pytest.mark.parametrize("name", ["qwen_16k", "qwen_32k_k1024", "qwen_32k_k4096",
+                                  "qwen_32k_k8192", "qwen_128k", "ragged_4"])
 def test_attention_full_size_sampled(oracle, name):
     w = gen.WORKLOADS[name]
     lens = w.kept_lengths()
@@ -151,6 +153,27 @@ def test_attention_full_size_sampled(oracle, name):
     rows = sample_rows(M, cu, n_random=24, seed=M)
     _attn_case(oracle, lens, w.n_q_heads, w.n_kv_heads, w.head_dim, "bf16", tg.ALGO_TCGEN05,
                seed=w.seed, rows=rows)
+
+
+@pytest.mark.parametrize("name", ["qwen_32k_k8192"])
+def test_ungated_full_n_attention_sampled(oracle, name):
+    """The ungated comparison of the 32k configuration: plain causal GQA
+    attention over all N tokens (no log-gates, gain 0, temperature 1), checked
+    on about a thousand query rows spread over the whole length."""
+    w = gen.WORKLOADS[name]
+    N = w.total_tokens
+    cu, q, k, v, _, _, _ = gen.attention_inputs([N], w.n_q_heads, w.n_kv_heads, w.head_dim,
+                                                w.seed + 5, "bf16", False)
+    Hq = w.n_q_heads
+    gain, temp = torch.zeros(Hq), torch.ones(Hq)
+    out, lse = tg.gated_attention(dev(q), dev(k), dev(v), cu, None, dev(gain), dev(temp),
+                                  want_lse=True)
+    rows = sample_rows(N, cu, n_random=1000, seed=N)
+    ref, ref_lse = oracle.gated_attention(q.float().numpy(), k.float().numpy(),
+                                          v.float().numpy(), cu, None, gain.numpy(),
+                                          temp.numpy(), rows=rows)
+    assert_close("ungated out", host_f32(out)[rows], ref, *ATTN_BF16)
+    assert_close("ungated lse", lse.cpu().numpy().T[rows], ref_lse, LSE_ATOL, 0.0)
 
 
 def test_attention_repeated_calls_identical():

@@ -3,7 +3,10 @@ allocate device memory (for example a server whose allocator owns the whole
 GPU, or code that must not allocate around CUDA-graph capture).  It takes the
 scratch of the key-range split from an array built into the library instead of
 a caller workspace.  Its results must match tg_gated_attention with a
-workspace, call after call.  This file is collected last on purpose."""
+workspace, call after call.  Some cases below split (their plan needs scratch,
+so the built-in array and the reset of its counters are exercised); one needs
+more than the array's 32 MiB and must run the unsplit plan instead.  This file
+is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -28,9 +31,22 @@ def _noalloc(q, k, v, cu, ls, gain, temp, out, lse):
     assert st == 0, (L.tg_status_string(st), L.tg_last_error_message())
 
 
+SCRATCH_BYTES = 32 << 20
+CASES = [([1000], 16, 8), ([2304], 16, 8), ([5, 0, 260, 1, 640], 16, 8), ([8448], 16, 8),
+         ([1280], 12, 4), ([2304], 12, 4), ([15000], 4, 2)]
+
+
+def test_cases_cover_split_and_oversize_plans():
+    """Host-only: the planner sizes these cases the same way on any machine with
+    148 SMs (a B200; the host planner assumes 148 without a device)."""
+    need = [tg.attention_workspace_bytes(np.array([0, *np.cumsum(l)], np.int32), hq, hkv, 128)
+            for l, hq, hkv in CASES]
+    assert any(0 < n <= SCRATCH_BYTES for n in need), need
+    assert any(n > SCRATCH_BYTES for n in need), need
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("lens,Hq,Hkv", [([1000], 16, 8), ([2304], 16, 8), ([5, 0, 260, 1, 640], 16, 8),
-                                         ([8448], 16, 8), ([1280], 12, 4), ([2304], 12, 4)])
+@pytest.mark.parametrize("lens,Hq,Hkv", CASES)
 def test_noalloc_matches_workspace_call_twice(lens, Hq, Hkv):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
