@@ -154,6 +154,57 @@ TG_API tg_status tg_topk_select(const float* z, int32_t batch, const int32_t* cu
                          const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
                          tg_stream_t stream);
 
+/*
+ * Bytes of the top-K workspace for a batch of `batch` prompts (0 outside
+ * 1..TG_MAX_BATCH): per prompt, the first radix pass's 2048-bin histogram of
+ * its document scores and a tag (8448 bytes).  total_tokens does not change
+ * the size.  The workspace carries the histograms from tg_gate_score_hist to
+ * tg_topk_select_ws; the caller zeroes it once after allocating it (for
+ * example cudaMemsetAsync), and every tg_topk_select_ws leaves it zeroed
+ * again.  Host-only.
+ */
+TG_API size_t tg_topk_workspace_bytes(int32_t batch, int64_t total_tokens);
+
+/*
+ * Step 1 with the selection's first radix pass folded into the gate's epilogue
+ * (the scores are in registers there): as tg_gate_score, and each document
+ * token's score is also counted into its prompt's first-pass histogram in the
+ * top-K workspace, so tg_topk_select_ws starts at the second pass.
+ *   batch, cu_seqlens_h[batch+1], doc_begin_h/doc_end_h[batch]: host, as for
+ *       tg_topk_select (cu_seqlens_h[batch] must equal n_tokens; 1..TG_MAX_BATCH
+ *       prompts)
+ *   topk_workspace, topk_workspace_bytes: device, >= tg_topk_workspace_bytes,
+ *       16-byte aligned, zero on entry (it is after allocation plus a memset
+ *       and after every tg_topk_select_ws); TG_ERR_WORKSPACE when smaller
+ * Other arguments and errors as tg_gate_score.  The histograms name the
+ * scores they were counted from (z_out): a tg_topk_select_ws on other scores,
+ * or on a workspace counted twice, finds the name or the counts wrong and
+ * counts the first pass itself.
+ */
+TG_API tg_status tg_gate_score_hist(const void* h, tg_dtype dtype, int64_t n_tokens,
+                                    int32_t d_model, const void* W1, const float* b1,
+                                    int32_t d_hidden, const float* w2, float b2, float* z_out,
+                                    int32_t batch, const int32_t* cu_seqlens_h,
+                                    const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                                    void* topk_workspace, size_t topk_workspace_bytes,
+                                    int32_t algo, tg_stream_t stream);
+
+/*
+ * Step 2 on a top-K workspace: the selection of tg_topk_select, exactly (the
+ * same rows), taking the first pass's histograms from the workspace when
+ * tg_gate_score_hist counted them from these scores z (otherwise counting
+ * them itself), and leaving the workspace zeroed for the next gate.
+ *   workspace, workspace_bytes: device, >= tg_topk_workspace_bytes(batch, .),
+ *       16-byte aligned (TG_ERR_WORKSPACE when smaller); calls that share a
+ *       workspace must not overlap on the GPU.
+ * Other arguments, order, limits and errors as tg_topk_select.
+ */
+TG_API tg_status tg_topk_select_ws(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                                   const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                                   const int32_t* budget_h, int32_t* kept_idx_out,
+                                   int32_t* cu_kept_out, void* workspace, size_t workspace_bytes,
+                                   tg_stream_t stream);
+
 #define TG_MAX_BUDGETS 8
 
 /*

@@ -26,6 +26,7 @@ __all__ = [
     "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
     "attention_kernel", "topk_select_multi", "random_select", "gated_attention_backward",
     "attention_backward_workspace_bytes", "rmsnorm", "qkv_rope_emit", "swiglu", "gated_delta_scan",
+    "topk_workspace_bytes", "topk_workspace",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -43,6 +44,7 @@ EXPORTED_SYMBOLS = (
     "tg_gated_attention_noalloc", "tg_topk_select_multi", "tg_random_select",
     "tg_gated_attention_backward", "tg_attention_backward_workspace_bytes", "tg_rmsnorm",
     "tg_qkv_rope_emit", "tg_swiglu", "tg_gated_delta_scan", "tg_last_device_error",
+    "tg_topk_workspace_bytes", "tg_gate_score_hist", "tg_topk_select_ws",
 )
 MAX_BUDGETS = 8
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
@@ -86,6 +88,12 @@ def library():
     L.tg_gate_score.argtypes = [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, _i32, _vp, _f32, _vp,
                                 _i32, _vp]
     L.tg_topk_select.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp]
+    L.tg_topk_workspace_bytes.argtypes = [_i32, _i64]
+    L.tg_gate_score_hist.argtypes = [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, _i32, _vp, _f32,
+                                     _vp, _i32, _i32p, _i32p, _i32p, _vp, ctypes.c_size_t, _i32,
+                                     _vp]
+    L.tg_topk_select_ws.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp,
+                                    ctypes.c_size_t, _vp]
     L.tg_topk_select_multi.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32, _i32p,
                                        ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp]
     L.tg_random_select.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp]
@@ -112,8 +120,10 @@ def library():
     L.tg_gated_delta_scan.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _i32, _i32p, _i32, _i32,
                                       _f32, _vp, _vp, _vp]
     for name in EXPORTED_SYMBOLS:
-        if name not in ("tg_status_string", "tg_last_error_message", "tg_version"):
+        if name not in ("tg_status_string", "tg_last_error_message", "tg_version",
+                        "tg_topk_workspace_bytes"):
             getattr(L, name).restype = ctypes.c_int
+    L.tg_topk_workspace_bytes.restype = ctypes.c_size_t
     _lib = L
     return L
 
@@ -190,8 +200,23 @@ def kept_offsets(cu_seqlens, doc_begin, doc_end, budget) -> np.ndarray:
     return out
 
 
-def gate_score(h, W1, b1, w2, b2, out=None, algo=ALGO_AUTO):
-    """z = w2 . GELU(W1 h + b1) + b2 for every row of h [n, d]."""
+def topk_workspace_bytes(batch, total_tokens=0):
+    """Bytes of the top-K workspace (first-pass histograms) for `batch` prompts."""
+    return int(library().tg_topk_workspace_bytes(int(batch), int(total_tokens)))
+
+
+def topk_workspace(batch, device=None):
+    """A zeroed top-K workspace for `batch` prompts (uint8 device tensor)."""
+    return torch.zeros(topk_workspace_bytes(batch), dtype=torch.uint8, device=device or "cuda")
+
+
+def gate_score(h, W1, b1, w2, b2, out=None, algo=ALGO_AUTO, topk_ws=None, cu_seqlens=None,
+               doc_begin=None, doc_end=None):
+    """z = w2 . GELU(W1 h + b1) + b2 for every row of h [n, d].
+
+    With ``topk_ws`` (a zeroed top-K workspace) and the prompt spans, the gate
+    also counts the selection's first radix pass into it (tg_gate_score_hist),
+    for a following ``topk_select(..., workspace=topk_ws)``."""
     n, d = h.shape
     dg = W1.shape[0]
     if W1.shape[1] != d or W1.dtype != h.dtype:
@@ -204,15 +229,28 @@ def gate_score(h, W1, b1, w2, b2, out=None, algo=ALGO_AUTO):
     _need_cuda(h, W1, b1, w2)
     if out is None:
         out = torch.empty(n, dtype=torch.float32, device=h.device)
-    _check("tg_gate_score", library().tg_gate_score(
+    if topk_ws is None:
+        _check("tg_gate_score", library().tg_gate_score(
+            _ptr(h), _dtype_code(h), n, d, _ptr(W1), _ptr(b1), dg, _ptr(w2), float(b2),
+            _ptr(out), algo, _stream(h.device)))
+        return out
+    if topk_ws.dtype != torch.uint8 or not topk_ws.is_contiguous() or topk_ws.device != h.device:
+        raise ValueError("topk_ws must be a contiguous uint8 tensor on h's device")
+    cu, cu_p = _host_i32(cu_seqlens)
+    s, s_p = _host_i32(doc_begin)
+    e, e_p = _host_i32(doc_end)
+    _check("tg_gate_score_hist", library().tg_gate_score_hist(
         _ptr(h), _dtype_code(h), n, d, _ptr(W1), _ptr(b1), dg, _ptr(w2), float(b2), _ptr(out),
-        algo, _stream(h.device)))
+        len(s), cu_p, s_p, e_p, _ptr(topk_ws), topk_ws.numel(), algo, _stream(h.device)))
     return out
 
 
-def topk_select(z, cu_seqlens, doc_begin, doc_end, budget, kept_idx=None, cu_kept=None):
+def topk_select(z, cu_seqlens, doc_begin, doc_end, budget, kept_idx=None, cu_kept=None,
+                workspace=None):
     """Per-prompt top-K of the document span (question kept).
 
+    ``workspace``: a top-K workspace, possibly holding the gate's first-pass
+    histograms of these scores (tg_topk_select_ws); left zeroed.
     Returns (kept_idx [M] int32 device, cu_kept [B+1] int32 device, cu_kept_host).
     """
     cu, cu_p = _host_i32(cu_seqlens)
@@ -224,15 +262,22 @@ def topk_select(z, cu_seqlens, doc_begin, doc_end, budget, kept_idx=None, cu_kep
     _expect("z", z, (int(cu[-1]),), torch.float32, z.device)
     _expect("kept_idx", kept_idx, (M,), torch.int32, z.device)
     _expect("cu_kept", cu_kept, (len(s) + 1,), torch.int32, z.device)
+    if workspace is not None and (workspace.dtype != torch.uint8 or
+                                  not workspace.is_contiguous() or workspace.device != z.device):
+        raise ValueError("workspace must be a contiguous uint8 tensor on z's device")
     _need_cuda(z)
     if kept_idx is None:
         kept_idx = torch.empty(max(M, 1), dtype=torch.int32, device=z.device)[:M]
     if cu_kept is None:
         cu_kept = torch.empty(len(s) + 1, dtype=torch.int32, device=z.device)
-    _expect("kept_idx", kept_idx, (M,), torch.int32, z.device)
-    _expect("cu_kept", cu_kept, (len(s) + 1,), torch.int32, z.device)
-    _check("tg_topk_select", library().tg_topk_select(
-        _ptr(z), len(s), cu_p, s_p, e_p, k_p, _ptr(kept_idx), _ptr(cu_kept), _stream(z.device)))
+    if workspace is None:
+        _check("tg_topk_select", library().tg_topk_select(
+            _ptr(z), len(s), cu_p, s_p, e_p, k_p, _ptr(kept_idx), _ptr(cu_kept),
+            _stream(z.device)))
+    else:
+        _check("tg_topk_select_ws", library().tg_topk_select_ws(
+            _ptr(z), len(s), cu_p, s_p, e_p, k_p, _ptr(kept_idx), _ptr(cu_kept), _ptr(workspace),
+            workspace.numel(), _stream(z.device)))
     return kept_idx, cu_kept, host
 
 
@@ -550,9 +595,14 @@ def gated_delta_scan(q, k, v, cu_kept_host, log_alpha, beta, eps=1e-6, out=None,
 
 def gated_prefill(h, q, k, v, W1, b1, w2, b2, gain, temp, cu_seqlens, doc_begin, doc_end,
                   budget, rope_theta=1e6, algo=ALGO_AUTO, want_lse=False):
-    """One gated layer: score, select, compact, attend.  Returns a dict of device tensors."""
-    z = gate_score(h, W1, b1, w2, b2, algo=algo)
-    kept_idx, cu_kept, cu_kept_host = topk_select(z, cu_seqlens, doc_begin, doc_end, budget)
+    """One gated layer: score (with the selection's first radix pass), select,
+    compact, attend.  Returns a dict of device tensors."""
+    B = len(np.asarray(doc_begin))
+    ws = topk_workspace(B, device=h.device) if B > 0 else None
+    z = gate_score(h, W1, b1, w2, b2, algo=algo, topk_ws=ws, cu_seqlens=cu_seqlens,
+                   doc_begin=doc_begin, doc_end=doc_end)
+    kept_idx, cu_kept, cu_kept_host = topk_select(z, cu_seqlens, doc_begin, doc_end, budget,
+                                                  workspace=ws)
     Hq, dh = q.shape[1], q.shape[2]
     (h_c, q_c, k_c, v_c), logsig = compact_gather(
         kept_idx, cu_seqlens, doc_begin, doc_end, budget, [h, q, k, v],

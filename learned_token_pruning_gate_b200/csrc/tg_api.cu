@@ -249,9 +249,11 @@ tg_status tg_kept_offsets(int32_t batch, const int32_t* cu, const int32_t* s, co
   return TG_OK;
 }
 
-tg_status tg_gate_score(const void* h, tg_dtype dtype, int64_t n_tokens, int32_t d_model,
-                        const void* W1, const float* b1, int32_t d_hidden, const float* w2,
-                        float b2, float* z_out, int32_t algo, tg_stream_t stream) {
+// The gate call with or without the top-K workspace's histograms.
+static tg_status gate_score_impl(const void* h, tg_dtype dtype, int64_t n_tokens, int32_t d_model,
+                                 const void* W1, const float* b1, int32_t d_hidden,
+                                 const float* w2, float b2, float* z_out, int32_t algo,
+                                 const GateHist& gh, tg_stream_t stream) {
   if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
   if (n_tokens < 0 || d_model <= 0 || d_hidden <= 0)
     return set_error(TG_ERR_INVALID_ARG, "n_tokens=%lld d_model=%d d_hidden=%d",
@@ -271,14 +273,69 @@ tg_status tg_gate_score(const void* h, tg_dtype dtype, int64_t n_tokens, int32_t
     return set_error(TG_ERR_UNSUPPORTED,
                      "tcgen05 gate needs bf16, d_model%%64==0, d_hidden in 32..256 step 32");
   if (algo == TG_ALGO_SIMT || !tc_ok)
-    return launch_gate_simt(h, dtype, n_tokens, d_model, W1, b1, d_hidden, w2, b2, z_out, st);
-  return launch_gate_tc(h, n_tokens, d_model, W1, b1, d_hidden, w2, b2, z_out, st);
+    return launch_gate_simt(h, dtype, n_tokens, d_model, W1, b1, d_hidden, w2, b2, z_out, gh, st);
+  return launch_gate_tc(h, n_tokens, d_model, W1, b1, d_hidden, w2, b2, z_out, gh, st);
 }
 
-tg_status tg_topk_select(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
-                         const int32_t* doc_begin_h, const int32_t* doc_end_h,
-                         const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
-                         tg_stream_t stream) {
+tg_status tg_gate_score(const void* h, tg_dtype dtype, int64_t n_tokens, int32_t d_model,
+                        const void* W1, const float* b1, int32_t d_hidden, const float* w2,
+                        float b2, float* z_out, int32_t algo, tg_stream_t stream) {
+  static thread_local GateHist none;  // hist = nullptr: no histogram
+  none.hist = nullptr;
+  return gate_score_impl(h, dtype, n_tokens, d_model, W1, b1, d_hidden, w2, b2, z_out, algo, none,
+                         stream);
+}
+
+size_t tg_topk_workspace_bytes(int32_t batch, int64_t total_tokens) {
+  (void)total_tokens;  // the histograms are per prompt, whatever its length
+  if (batch <= 0 || batch > kMaxBatch) return 0;
+  return static_cast<size_t>(batch) * kHistStride * sizeof(uint32_t);
+}
+
+static tg_status check_topk_workspace(int32_t batch, const void* ws, size_t bytes) {
+  if (!ws) return set_error(TG_ERR_INVALID_ARG, "top-K workspace is null");
+  if (!aligned16(ws)) return set_error(TG_ERR_ALIGNMENT, "top-K workspace must be 16-byte aligned");
+  const size_t need = tg_topk_workspace_bytes(batch, 0);
+  if (bytes < need)
+    return set_error(TG_ERR_WORKSPACE, "top-K workspace: %zu bytes given, %zu needed", bytes, need);
+  return TG_OK;
+}
+
+tg_status tg_gate_score_hist(const void* h, tg_dtype dtype, int64_t n_tokens, int32_t d_model,
+                             const void* W1, const float* b1, int32_t d_hidden, const float* w2,
+                             float b2, float* z_out, int32_t batch, const int32_t* cu_seqlens_h,
+                             const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                             void* topk_workspace, size_t topk_workspace_bytes, int32_t algo,
+                             tg_stream_t stream) {
+  static const int32_t kNoBudget[kMaxBatch] = {};  // the spans only: budgets play no part here
+  PromptTable t;
+  tg_status r = build_table(batch, cu_seqlens_h, doc_begin_h, doc_end_h, kNoBudget, &t, nullptr,
+                            nullptr);
+  if (r != TG_OK) return r;
+  if (batch == 0) return set_error(TG_ERR_INVALID_ARG, "the histograms need at least one prompt");
+  if (t.start[batch] != n_tokens)
+    return set_error(TG_ERR_SHAPE, "cu_seqlens ends at %d, n_tokens=%lld", t.start[batch],
+                     static_cast<long long>(n_tokens));
+  if ((r = check_topk_workspace(batch, topk_workspace, topk_workspace_bytes)) != TG_OK) return r;
+  static thread_local GateHist gh;
+  gh.hist = static_cast<uint32_t*>(topk_workspace);
+  gh.z = z_out;
+  gh.n = static_cast<int32_t>(n_tokens);
+  gh.batch = batch;
+  for (int b = 0; b <= batch; ++b) gh.start[b] = t.start[b];
+  for (int b = 0; b < batch; ++b) {
+    gh.doc_lo[b] = t.start[b] + t.doc_begin[b];
+    gh.doc_hi[b] = t.start[b] + t.doc_end[b];
+  }
+  return gate_score_impl(h, dtype, n_tokens, d_model, W1, b1, d_hidden, w2, b2, z_out, algo, gh,
+                         stream);
+}
+
+// The selection with or without the gate's histograms.
+static tg_status topk_select_impl(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                                  const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                                  const int32_t* budget_h, int32_t* kept_idx_out,
+                                  int32_t* cu_kept_out, uint32_t* hist, tg_stream_t stream) {
   PromptTable t;
   int max_len = 0;
   tg_status r = build_table(batch, cu_seqlens_h, doc_begin_h, doc_end_h, budget_h, &t, &max_len,
@@ -290,8 +347,28 @@ tg_status tg_topk_select(const float* z, int32_t batch, const int32_t* cu_seqlen
   if (t.start[batch] > 0 && !z) return set_error(TG_ERR_INVALID_ARG, "z is null");
   if (max_len > 360448)
     return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens exceeds 360448", max_len);
-  return launch_topk(z, nullptr, &t, 1, max_len, &kept_idx_out, &cu_kept_out,
+  return launch_topk(z, nullptr, &t, 1, max_len, &kept_idx_out, &cu_kept_out, hist,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+tg_status tg_topk_select(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                         const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                         const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
+                         tg_stream_t stream) {
+  return topk_select_impl(z, batch, cu_seqlens_h, doc_begin_h, doc_end_h, budget_h, kept_idx_out,
+                          cu_kept_out, nullptr, stream);
+}
+
+tg_status tg_topk_select_ws(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                            const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                            const int32_t* budget_h, int32_t* kept_idx_out, int32_t* cu_kept_out,
+                            void* workspace, size_t workspace_bytes, tg_stream_t stream) {
+  if (batch > 0 && batch <= kMaxBatch) {
+    tg_status r = check_topk_workspace(batch, workspace, workspace_bytes);
+    if (r != TG_OK) return r;
+  }
+  return topk_select_impl(z, batch, cu_seqlens_h, doc_begin_h, doc_end_h, budget_h, kept_idx_out,
+                          cu_kept_out, static_cast<uint32_t*>(workspace), stream);
 }
 
 tg_status tg_topk_select_multi(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
@@ -316,7 +393,7 @@ tg_status tg_topk_select_multi(const float* z, int32_t batch, const int32_t* cu_
   if (t[0].start[batch] > 0 && !z) return set_error(TG_ERR_INVALID_ARG, "z is null");
   if (max_len > 360448)
     return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens exceeds 360448", max_len);
-  return launch_topk(z, nullptr, t, n_budgets, max_len, kept_idx_out, cu_kept_out,
+  return launch_topk(z, nullptr, t, n_budgets, max_len, kept_idx_out, cu_kept_out, nullptr,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -335,7 +412,7 @@ tg_status tg_random_select(const uint32_t* keys, int32_t batch, const int32_t* c
   if (t.start[batch] > 0 && !keys) return set_error(TG_ERR_INVALID_ARG, "keys is null");
   if (max_len > 360448)
     return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens exceeds 360448", max_len);
-  return launch_topk(nullptr, keys, &t, 1, max_len, &kept_idx_out, &cu_kept_out,
+  return launch_topk(nullptr, keys, &t, 1, max_len, &kept_idx_out, &cu_kept_out, nullptr,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -14,6 +14,12 @@
 //              the next tile's MMAs overlap this epilogue.
 // gate_simt_kernel is the CUDA-core path for fp32 and for shapes the tensor-core
 // kernel does not take.
+//
+// With a top-K workspace (tg_gate_score_hist) every kernel's epilogue also
+// counts each document token's score into its prompt's first radix-pass
+// histogram (top 11 bits of the order key), so the top-K select starts at its
+// second pass: the scores are in registers here anyway, and the histogram costs
+// one global atomic per distinct bin of a warp's rows.
 #include "tg_internal.cuh"
 
 namespace tg {
@@ -73,10 +79,12 @@ __global__ void __launch_bounds__(256) gate_simt_kernel(const T* __restrict__ h,
                                                         const T* __restrict__ W1,
                                                         const float* __restrict__ b1, int dg,
                                                         const float* __restrict__ w2, float b2,
-                                                        float* __restrict__ z) {
+                                                        float* __restrict__ z,
+                                                        const __grid_constant__ GateHist gh) {
   const int lane = threadIdx.x & 31;
   grid_dep_wait();
   grid_dep_launch();
+  gate_hist_tags(gh, 0, blockDim.x);
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t j = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        j < n; j += warps) {
@@ -91,6 +99,7 @@ __global__ void __launch_bounds__(256) gate_simt_kernel(const T* __restrict__ h,
       zsum = fmaf(__ldg(w2 + u), gelu_erf(acc + __ldg(b1 + u)), zsum);
     }
     if (lane == 0) z[j] = zsum + b2;
+    if (gh.hist) gate_hist_add(gh, static_cast<int>(j), zsum + b2, lane == 0);
   }
 }
 
@@ -130,7 +139,7 @@ struct GateSmemLayout {
 
 __global__ void __launch_bounds__(kThreads, 1)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
-                   const __grid_constant__ GateTcParams p) {
+                   const __grid_constant__ GateTcParams p, const __grid_constant__ GateHist gh) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -169,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_b1[i] = p.b1[i];
       s_w2[i] = p.w2[i];
     }
+    gate_hist_tags(gh, 64, 128);
   }
   tc_fence_before();
   __syncthreads();
@@ -254,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(10 + acc));
       const int row = tile * kBM + row_local;
       if (row < p.n) p.z[row] = sum + p.b2;
+      if (gh.hist) gate_hist_add(gh, row, sum + p.b2, row < p.n);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -300,7 +311,7 @@ struct Gate2Layout {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     gate_tc2_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
-                    const __grid_constant__ GateTcParams p) {
+                    const __grid_constant__ GateTcParams p, const __grid_constant__ GateHist gh) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -423,6 +434,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       s_b1[i] = p.b1[i];
       s_w2[i] = p.w2[i];
     }
+    gate_hist_tags(gh, 64, 256);
     named_barrier(2, 256);
     uint32_t acc = 0, acc_phase = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs) {
@@ -442,7 +454,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       if (half) s_part[acc * 128 + row_local] = sum;
       named_barrier(1, 256);  // both halves of every row are summed
       const int row = tile * 2 * kBM + static_cast<int>(rank) * kBM + row_local;
-      if (!half && row < p.n) p.z[row] = sum + s_part[acc * 128 + row_local] + p.b2;
+      if (!half) {
+        const float zr = sum + s_part[acc * 128 + row_local] + p.b2;
+        if (row < p.n) p.z[row] = zr;
+        if (gh.hist) gate_hist_add(gh, row, zr, row < p.n);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -461,7 +477,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 
 tg_status launch_gate_simt(const void* h, tg_dtype dt, int64_t n, int d, const void* W1,
                            const float* b1, int dg, const float* w2, float b2, float* z,
-                           cudaStream_t st) {
+                           const GateHist& gh, cudaStream_t st) {
   const int64_t warps_needed = n;
   int64_t blocks = (warps_needed + 7) / 8;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
@@ -469,15 +485,16 @@ tg_status launch_gate_simt(const void* h, tg_dtype dt, int64_t n, int d, const v
   if (dt == TG_BF16)
     gate_simt_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(h), n, d, static_cast<const __nv_bfloat16*>(W1), b1, dg,
-        w2, b2, z);
+        w2, b2, z, gh);
   else
     gate_simt_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        static_cast<const float*>(h), n, d, static_cast<const float*>(W1), b1, dg, w2, b2, z);
+        static_cast<const float*>(h), n, d, static_cast<const float*>(W1), b1, dg, w2, b2, z, gh);
   return cuda_check(cudaGetLastError(), "gate_simt launch");
 }
 
 tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const float* b1, int dg,
-                         const float* w2, float b2, float* z, cudaStream_t st) {
+                         const float* w2, float b2, float* z, const GateHist& gh,
+                         cudaStream_t st) {
   CUtensorMap tm_h, tm_w;
   // CTA-pair kernel (each CTA stages half of W1) when the 128-column stages tile d
   const bool pairs = num_sms() >= 2 && d % kBK2 == 0;
@@ -508,7 +525,7 @@ tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const 
     if (r2 != TG_OK) return r2;
     int npairs = num_sms() / 2;
     if (npairs > p.num_tiles) npairs = p.num_tiles;
-    gate_tc2_kernel<<<2 * npairs, kThreads2, smem2, st>>>(tm_h, tm_w, p);
+    gate_tc2_kernel<<<2 * npairs, kThreads2, smem2, st>>>(tm_h, tm_w, p, gh);
     return cuda_check(cudaGetLastError(), "gate_tc2 launch");
   }
   p.num_tiles = static_cast<int32_t>((n + kBM - 1) / kBM);
@@ -521,7 +538,7 @@ tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const 
   if (r != TG_OK) return r;
   int grid = num_sms();
   if (grid > p.num_tiles) grid = p.num_tiles;
-  gate_tc_kernel<<<grid, kThreads, smem, st>>>(tm_h, tm_w, p);
+  gate_tc_kernel<<<grid, kThreads, smem, st>>>(tm_h, tm_w, p, gh);
   return cuda_check(cudaGetLastError(), "gate_tc launch");
 }
 

@@ -27,6 +27,25 @@ struct PromptTable {
   int32_t kept_start[kMaxBatch + 1];  // cu_kept
 };
 
+// First-pass radix histograms handed from the gate to the top-K select (the
+// top-K workspace).  Per prompt: kHistBins counts of the top 11 bits of the
+// order key (below) of its document tokens' scores, then a 4-word tag {magic,
+// total tokens, score pointer lo, hi} naming the scores they were counted from.
+constexpr int kHistBins = 2048;
+constexpr int kHistStride = 2112;  // words per prompt: 8448 bytes, a multiple of 256
+constexpr uint32_t kHistMagic = 0x7A6E5B1Fu;
+
+// What a gate launch needs to add its scores to the top-K workspace.
+struct GateHist {
+  uint32_t* hist;              // [batch][kHistStride] or null (no histogram)
+  const float* z;              // the scores the gate writes (for the tag)
+  int32_t n;                   // total tokens (for the tag)
+  int32_t batch;
+  int32_t start[kMaxBatch + 1];  // cu_seqlens
+  int32_t doc_lo[kMaxBatch];     // absolute document span [doc_lo, doc_hi) of each prompt
+  int32_t doc_hi[kMaxBatch];
+};
+
 // Bits of the device status word.
 enum : uint32_t {
   kDevTimeoutGate = 1u << 0,
@@ -59,14 +78,17 @@ class SymbolAddressCache {
 int num_sms();
 
 // Kernel launchers (each validates nothing: the C ABI layer has done it).
+// The gate launchers add the first-pass histograms when gh.hist is non-null.
 tg_status launch_gate_simt(const void* h, tg_dtype dt, int64_t n, int d, const void* W1,
                            const float* b1, int dg, const float* w2, float b2, float* z,
-                           cudaStream_t st);
+                           const GateHist& gh, cudaStream_t st);
 tg_status launch_gate_tc(const void* h, int64_t n, int d, const void* W1, const float* b1, int dg,
-                         const float* w2, float b2, float* z, cudaStream_t st);
+                         const float* w2, float b2, float* z, const GateHist& gh,
+                         cudaStream_t st);
+// hist: the top-K workspace of a single-budget score selection, or null.
 tg_status launch_topk(const float* z, const uint32_t* keys, const PromptTable* tables,
                       int n_budgets, int max_len, int32_t* const* kept_idx,
-                      int32_t* const* cu_kept, cudaStream_t st);
+                      int32_t* const* cu_kept, uint32_t* hist, cudaStream_t st);
 tg_status launch_gather(const int32_t* kept_idx, int64_t m_total, const PromptTable& pt,
                         tg_dtype dt, const tg_gather_tensor* tensors, int n_tensors, int head_dim,
                         double theta, const float* z, float* logsig, cudaStream_t st);
@@ -107,6 +129,51 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uin
                          uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 
 #if defined(__CUDACC__)
+
+// Order-preserving key of an fp32 score: larger score -> larger key; -0.0 maps
+// to +0.0; NaN maps to 0, below every number (-inf maps to 0x007FFFFF).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0u;
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Adds one score to its prompt's first-pass histogram when the row is a
+// document token.  The warp's converged lanes call it together (active: the
+// lane holds a row); lanes that hit the same bin add once, together.
+__device__ __forceinline__ void gate_hist_add(const GateHist& gh, int row, float z, bool active) {
+  uint32_t idx = 0xFFFFFFFFu;
+  if (active) {
+    int lo = 0, hi = gh.batch - 1;  // the prompt: last b with start[b] <= row
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (gh.start[mid] <= row) lo = mid;
+      else hi = mid - 1;
+    }
+    if (row >= gh.doc_lo[lo] && row < gh.doc_hi[lo])
+      idx = static_cast<uint32_t>(lo) * kHistStride + (order_key(z) >> 21);
+  }
+  const unsigned mask = __ballot_sync(__activemask(), idx != 0xFFFFFFFFu);
+  if (idx != 0xFFFFFFFFu) {
+    const unsigned peers = __match_any_sync(mask, idx);
+    if (static_cast<int>(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(gh.hist + idx, __popc(peers));
+  }
+}
+
+// The tag of every prompt's histogram (written once per gate launch, by the
+// threads [first, first + stride) of block 0).
+__device__ __forceinline__ void gate_hist_tags(const GateHist& gh, int first, int stride) {
+  if (!gh.hist || blockIdx.x != 0) return;
+  const uint64_t zp = reinterpret_cast<uint64_t>(gh.z);
+  for (int b = static_cast<int>(threadIdx.x) - first; b >= 0 && b < gh.batch; b += stride) {
+    uint32_t* tag = gh.hist + static_cast<size_t>(b) * kHistStride + kHistBins;
+    tag[0] = kHistMagic;
+    tag[1] = static_cast<uint32_t>(gh.n);
+    tag[2] = static_cast<uint32_t>(zp);
+    tag[3] = static_cast<uint32_t>(zp >> 32);
+  }
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

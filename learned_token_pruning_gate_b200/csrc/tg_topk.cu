@@ -9,23 +9,26 @@
 // selector ablation): larger first, lower index on ties, in both cases.
 //  1. Each CTA caches its slice of the scores in shared memory as
 //     order-preserving 32-bit keys (padded by one word per 32 so both strided
-//     and per-thread-contiguous walks are free of bank conflicts) and builds the
-//     first radix histogram while loading.
+//     and per-thread-contiguous walks are free of bank conflicts).
 //  2. Up to three radix passes (11, 11, 10 bits) find the K-th largest key T;
 //     when every key of a pass's boundary bin is kept, the low bits cannot
 //     change the set and the search stops there (T then fixes only the high
-//     bits; usually the last pass is skipped for continuous scores).  Every
-//     cross-CTA step is a one-way write: each CTA adds its non-zero bins into
-//     the leader CTA's histogram with remote shared-memory atomics, a cluster
-//     barrier publishes them, the leader scans and pushes the chosen digit into
-//     every CTA's shared memory, and a second barrier publishes that.  No
-//     thread waits on a distributed-shared-memory read.
+//     bits; usually the last pass is skipped for continuous scores).
+//     The first pass's histogram comes from the gate when it counted these
+//     scores into the top-K workspace (tg_gate_score_hist): every CTA reads
+//     the prompt's 2048 bins and picks the digit itself, with no exchange.
+//     Otherwise, and for the later passes, each CTA adds its non-zero bins
+//     into every CTA's totals with remote shared-memory atomics, one cluster
+//     barrier publishes them, and every CTA scans its own copy, so all of them
+//     take the same digit without waiting on a leader.  No thread waits on a
+//     distributed-shared-memory read.
 //  3. Ordered compaction: thread t owns a contiguous run of keys; one packed
 //     block scan of (count of keys > T or protected, count of keys == T) gives
 //     every thread its output offset and its rank among the ties (CTA totals
 //     are pushed to the higher-ranked CTAs), so ties go to the lower index and
 //     the kept rows come out in ascending order.
-// The only waits are hardware barriers; no global scratch is used.
+// The only waits are hardware barriers.  The only global scratch is the
+// optional top-K workspace, which the call leaves zeroed for the next gate.
 #include <cooperative_groups.h>
 
 #include "tg_internal.cuh"
@@ -36,7 +39,7 @@ namespace tg {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr int kBins = 2048;
+constexpr int kBins = kHistBins;
 constexpr int kMaxCluster = 8;
 
 struct TopkParams {
@@ -48,17 +51,9 @@ struct TopkParams {
   const float* z;      // scores (kKeys = false)
   const uint32_t* keys;  // caller keys (kKeys = true)
   uint32_t* status;
-  int32_t cluster;  // CTAs per (budget, prompt)
+  uint32_t* hist;      // top-K workspace with the gate's first-pass histograms, or null
+  int32_t cluster;     // CTAs per (budget, prompt)
 };
-
-// Order-preserving key: larger score -> larger key; -0.0 maps to +0.0; NaN maps
-// to 0, below every number (-inf maps to 0x007FFFFF).
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0u;
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 __host__ __device__ __forceinline__ int padded(int i) { return i + (i >> 5); }
 
@@ -93,11 +88,45 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
   return r;
 }
 
+// Run by every thread of a CTA over one pass's totals tot[0, nb): the digit d
+// whose bin holds the k_rem-th largest key, i.e. the keys of larger digits
+// number fewer than k_rem and those of digits >= d at least k_rem.  Writes
+// (d, keys above d, keys in d's bin) to s_sel, zeroes tot for a later pass and
+// returns the totals' sum.  Thread t owns bins nb-1-t*bpt-j (descending digit
+// order), so an exclusive scan counts the larger digits.
+__device__ uint32_t select_digit(uint32_t* tot, uint32_t nb, uint32_t k_rem, uint32_t* s_scan,
+                                 uint32_t* s_sel) {
+  const int tid = threadIdx.x;
+  const uint32_t bpt = nb / kThreads;  // 2 or 1
+  uint32_t cnt[2] = {0, 0};
+  for (uint32_t j = 0; j < bpt; ++j) {
+    const uint32_t bin = nb - 1 - tid * bpt - j;
+    cnt[j] = tot[bin];
+    tot[bin] = 0;
+  }
+  const uint32_t mine = cnt[0] + cnt[1];
+  uint32_t total = 0;
+  uint32_t above = block_excl_scan(mine, s_scan, &total);
+  if (above < k_rem && above + mine >= k_rem) {
+    for (uint32_t j = 0; j < bpt; ++j) {
+      if (above + cnt[j] >= k_rem) {
+        s_sel[0] = nb - 1 - tid * bpt - j;
+        s_sel[1] = above;
+        s_sel[2] = cnt[j];
+        break;
+      }
+      above += cnt[j];
+    }
+  }
+  __syncthreads();
+  return total;
+}
+
 template <bool kKeys>
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant__ TopkParams p) {
   extern __shared__ uint32_t s_keys[];  // padded layout
   __shared__ uint32_t s_hist[kBins];           // this CTA's histogram of the current pass
-  __shared__ uint32_t s_total[2][kBins];       // cluster totals (used in the leader only)
+  __shared__ uint32_t s_total[2][kBins];       // cluster totals (every CTA holds a copy)
   __shared__ uint32_t s_scan[33];
   __shared__ uint32_t s_sel[3];                // digit, count above, count in the digit's bin
   __shared__ uint32_t s_cnt[kMaxCluster][2];   // lower-ranked CTAs' (sure, tie) counts
@@ -126,88 +155,98 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
     s_total[1][i] = 0;
   }
   __syncthreads();
-  grid_dep_wait();  // the scores are complete
+  // this CTA's totals are zero: the others may add into them once the barrier
+  // completes (its wait comes after the scores are loaded)
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  grid_dep_wait();  // the scores (and the gate's histograms) are complete
   grid_dep_launch();
-  // keys into shared memory; pass-0 histogram (top 11 bits) on the way
+
+  // The gate's first-pass histogram of this prompt, when it counted these
+  // scores (the tag names them); the same decision in every CTA of the cluster.
+  uint32_t* hist_b = p.hist ? p.hist + static_cast<size_t>(b) * kHistStride : nullptr;
+  bool from_gate = false;
+  if (!kKeys && hist_b && mode == 2) {
+    const uint32_t* tag = hist_b + kBins;
+    const uint64_t zp = reinterpret_cast<uint64_t>(p.z);
+    from_gate = tag[0] == kHistMagic &&
+                tag[1] == static_cast<uint32_t>(p.pt.start[p.pt.batch]) &&
+                tag[2] == static_cast<uint32_t>(zp) && tag[3] == static_cast<uint32_t>(zp >> 32);
+    if (from_gate)
+      for (int i = tid; i < kBins; i += kThreads) s_hist[i] = __ldcg(hist_b + i);
+  }
+  // keys into shared memory; the first-pass histogram on the way when it is
+  // counted here
   for (int i = tid; i < len; i += kThreads) {
     const uint32_t key =
         kKeys ? __ldg(p.keys + start + lo + i) : order_key(__ldg(p.z + start + lo + i));
     s_keys[padded(i)] = key;
     const int32_t pos = lo + i;
-    if (mode == 2 && pos >= ds && pos < de) atomicAdd(&s_hist[key >> 21], 1u);
+    if (!from_gate && mode == 2 && pos >= ds && pos < de) atomicAdd(&s_hist[key >> 21], 1u);
   }
-  cluster.sync();  // every CTA has started and zeroed its totals
+  __syncthreads();
 
   uint32_t T = 0, need = 0;
   uint32_t hmask = 0xFFFFFFFFu;  // key bits the threshold T fixes
-  if (mode == 2) {
-    uint32_t* lead_sel = cluster.map_shared_rank(s_sel, 0);
-    uint32_t prefix = 0, k_rem = static_cast<uint32_t>(kk);
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const int nbits = pass == 2 ? 10 : 11;
-      const uint32_t nb = 1u << nbits;
-      if (pass > 0) {
-        const uint32_t high_mask = 0xFFFFFFFFu << (shift + nbits);
-        for (int i = tid; i < len; i += kThreads) {
-          const int32_t pos = lo + i;
-          if (pos < ds || pos >= de) continue;
-          const uint32_t key = s_keys[padded(i)];
-          if ((key & high_mask) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
-        }
-        __syncthreads();
-      }
-      // non-zero local bins into the leader's totals (one-way), local bins cleared
-      uint32_t* total = cluster.map_shared_rank(s_total[pass & 1], 0);
-      for (int i = tid; i < static_cast<int>(nb); i += kThreads) {
-        const uint32_t c = s_hist[i];
-        if (c) {
-          atomicAdd(total + i, c);
-          s_hist[i] = 0;
-        }
-      }
-      cluster.sync();  // totals complete in the leader
-      if (r == 0) {
-        // Thread t owns bins [nb-1 - t*bpt - (bpt-1), nb-1 - t*bpt]: thread order is
-        // descending digit order, so an exclusive scan counts the larger digits.
-        uint32_t* tot = s_total[pass & 1];
-        const uint32_t bpt = nb / kThreads;  // 2 or 1
-        uint32_t cnt[2] = {0, 0};
-        for (uint32_t j = 0; j < bpt; ++j) {
-          const uint32_t bin = nb - 1 - tid * bpt - j;
-          cnt[j] = tot[bin];
-          tot[bin] = 0;  // ready for pass + 2
-        }
-        const uint32_t mine = cnt[0] + cnt[1];
-        uint32_t above = block_excl_scan(mine, s_scan, nullptr);
-        if (above < k_rem && above + mine >= k_rem) {
-          for (uint32_t j = 0; j < bpt; ++j) {
-            if (above + cnt[j] >= k_rem) {
-              const uint32_t digit = nb - 1 - tid * bpt - j;
-              for (int rr = 0; rr < CL; ++rr) {  // push the choice to every CTA
-                uint32_t* sel = cluster.map_shared_rank(s_sel, rr);
-                sel[0] = digit;
-                sel[1] = above;
-                sel[2] = cnt[j];
-              }
-              break;
-            }
-            above += cnt[j];
-          }
-        }
-      }
-      cluster.sync();  // the chosen digit is visible everywhere
-      prefix |= s_sel[0] << shift;
+  uint32_t prefix = 0, k_rem = static_cast<uint32_t>(kk);
+  int pass = 0;
+  bool done = mode != 2;
+  if (from_gate) {
+    const uint32_t total = select_digit(s_hist, kBins, k_rem, s_scan, s_sel);  // clears s_hist
+    if (total == static_cast<uint32_t>(n_doc)) {
+      prefix = s_sel[0] << 21;
       k_rem -= s_sel[1];
-      if (s_sel[2] == k_rem) {
-        // every key of the boundary bin is kept: the remaining low bits cannot
-        // change the set, so stop here (the same decision in every CTA)
-        hmask = 0xFFFFFFFFu << shift;
-        break;
+      pass = 1;
+      if (s_sel[2] == k_rem) {  // the boundary bin is kept whole
+        hmask = 0xFFFFFFFFu << 21;
+        done = true;
+      }
+    } else {
+      // not the histogram of these scores after all: count the first pass here
+      for (int i = tid; i < len; i += kThreads) {
+        const int32_t pos = lo + i;
+        if (pos >= ds && pos < de) atomicAdd(&s_hist[s_keys[padded(i)] >> 21], 1u);
+      }
+      __syncthreads();
+    }
+  }
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // every CTA's totals are zero
+
+#pragma unroll 1
+  for (; !done && pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nbits = pass == 2 ? 10 : 11;
+    const uint32_t nb = 1u << nbits;
+    if (pass > 0) {
+      const uint32_t high_mask = 0xFFFFFFFFu << (shift + nbits);
+      for (int i = tid; i < len; i += kThreads) {
+        const int32_t pos = lo + i;
+        if (pos < ds || pos >= de) continue;
+        const uint32_t key = s_keys[padded(i)];
+        if ((key & high_mask) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
+      }
+      __syncthreads();
+    }
+    // non-zero local bins into every CTA's totals (one-way), local bins cleared
+    uint32_t* buf = s_total[pass & 1];
+    for (int i = tid; i < static_cast<int>(nb); i += kThreads) {
+      const uint32_t c = s_hist[i];
+      if (c) {
+        for (int rr = 0; rr < CL; ++rr) atomicAdd(cluster.map_shared_rank(buf, rr) + i, c);
+        s_hist[i] = 0;
       }
     }
-    (void)lead_sel;
+    cluster.sync();  // every CTA holds the cluster's totals of this pass
+    select_digit(buf, nb, k_rem, s_scan, s_sel);  // clears buf for pass + 2
+    prefix |= s_sel[0] << shift;
+    k_rem -= s_sel[1];
+    if (s_sel[2] == k_rem) {
+      // every key of the boundary bin is kept: the remaining low bits cannot
+      // change the set, so stop here (the same decision in every CTA)
+      hmask = 0xFFFFFFFFu << shift;
+      break;
+    }
+  }
+  if (mode == 2) {
     T = prefix;
     need = k_rem;  // how many keys whose fixed bits equal T to keep, lowest indices first
   }
@@ -263,13 +302,19 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
     p.cu_kept[q][b + 1] = p.kept_start[q][b + 1];
     if (b == 0) p.cu_kept[q][0] = 0;
   }
+  // leave the workspace zeroed for the next gate (every CTA read it before the
+  // barriers above); the tag is cleared so the bins are never reused
+  if (hist_b && r == 0) {
+    for (int i = tid; i < kBins; i += kThreads) hist_b[i] = 0;
+    if (tid == 0) hist_b[kBins] = 0;
+  }
 }
 
 }  // namespace
 
 tg_status launch_topk(const float* z, const uint32_t* keys, const PromptTable* tables,
                       int n_budgets, int max_len, int32_t* const* kept_idx,
-                      int32_t* const* cu_kept, cudaStream_t st) {
+                      int32_t* const* cu_kept, uint32_t* hist, cudaStream_t st) {
   static thread_local TopkParams p;  // ~11 KB: kept off the stack
   memset(&p, 0, sizeof(p));
   p.pt = tables[0];
@@ -281,6 +326,7 @@ tg_status launch_topk(const float* z, const uint32_t* keys, const PromptTable* t
   }
   p.z = z;
   p.keys = keys;
+  p.hist = (n_budgets == 1 && !keys) ? hist : nullptr;
   p.status = device_status_word();
   if (!p.status) return set_error(TG_ERR_CUDA, "device status word unavailable");
   const int cl = kMaxCluster;  // latency-bound: spread every prompt over 8 SMs

@@ -4,7 +4,9 @@
 (scores, kept indices, compacted residual/q/k/v, bias term, attention output)
 and holds every C-ABI argument pre-marshalled, so ``run()`` is exactly four
 library calls on one stream with no allocation and no host synchronisation --
-the form that CUDA-graph capture and per-kernel timing need.
+the form that CUDA-graph capture and per-kernel timing need.  The gate counts
+the selection's first radix pass into the layer's top-K workspace
+(tg_gate_score_hist), and the selection starts from it (tg_topk_select_ws).
 """
 from __future__ import annotations
 
@@ -15,7 +17,7 @@ import torch
 
 from . import (ALGO_AUTO, GatherTensor, _check, _dtype_code, _host_i32,
                attention_workspace_bytes, gated_attention, kept_offsets, library, qkv_rope_emit,
-               rmsnorm, swiglu)
+               rmsnorm, swiglu, topk_workspace_bytes)
 
 
 class GatedLayer:
@@ -53,6 +55,10 @@ class GatedLayer:
         ws = attention_workspace_bytes(self.cu_kept_host, self.Hq, self.Hkv, self.dh, q.dtype, algo)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
         self.ws_bytes = ws
+        # the top-K workspace: the gate counts the selection's first radix pass
+        # into it, the selection reads it and leaves it zeroed (zero to start)
+        self.topk_ws_bytes = topk_workspace_bytes(self.B) if self.B > 0 else 0
+        self.topk_ws = torch.zeros(max(self.topk_ws_bytes, 1), dtype=torch.uint8, device=dev)
         self.dcode = _dtype_code(h)
         self.tensors = (GatherTensor * 4)()
         for i, (src, dst, heads) in enumerate([(h, self.h_c, 0), (q, self.q_c, self.Hq),
@@ -65,22 +71,33 @@ class GatedLayer:
         self._p = {n: vp(t.data_ptr()) for n, t in dict(
             h=h, q=q, k=k, v=v, W1=W1, b1=b1, w2=w2, gain=gain, temp=temp, z=self.z,
             kept=self.kept_idx, cu_kept=self.cu_kept, q_c=self.q_c, k_c=self.k_c, v_c=self.v_c,
-            logsig=self.logsig, out=self.out).items()}
+            logsig=self.logsig, out=self.out, topk_ws=self.topk_ws).items()}
         self._p["ws"] = vp(self.workspace.data_ptr()) if self.workspace is not None else None
         self._p["lse"] = vp(self.lse.data_ptr()) if self.lse is not None else None
 
     # each step is one C-ABI call; `stream` is a raw cudaStream_t handle
     def gate(self, stream):
         p = self._p
-        _check("tg_gate_score", self.L.tg_gate_score(
+        if self.topk_ws_bytes == 0:
+            _check("tg_gate_score", self.L.tg_gate_score(
+                p["h"], self.dcode, self.N, self.d, p["W1"], p["b1"], self.dg, p["w2"], self.b2,
+                p["z"], self.algo, stream))
+            return
+        _check("tg_gate_score_hist", self.L.tg_gate_score_hist(
             p["h"], self.dcode, self.N, self.d, p["W1"], p["b1"], self.dg, p["w2"], self.b2,
-            p["z"], self.algo, stream))
+            p["z"], self.B, self.cu_p, self.s_p, self.e_p, p["topk_ws"], self.topk_ws_bytes,
+            self.algo, stream))
 
     def topk(self, stream):
         p = self._p
-        _check("tg_topk_select", self.L.tg_topk_select(
+        if self.topk_ws_bytes == 0:
+            _check("tg_topk_select", self.L.tg_topk_select(
+                p["z"], self.B, self.cu_p, self.s_p, self.e_p, self.k_p, p["kept"],
+                p["cu_kept"], stream))
+            return
+        _check("tg_topk_select_ws", self.L.tg_topk_select_ws(
             p["z"], self.B, self.cu_p, self.s_p, self.e_p, self.k_p, p["kept"], p["cu_kept"],
-            stream))
+            p["topk_ws"], self.topk_ws_bytes, stream))
 
     def gather(self, stream):
         p = self._p

@@ -330,3 +330,31 @@ def test_delta_scan_wrapper_rejects_mismatched_shapes():
         tg.gated_delta_scan(x, x, x, [0, 6], a.double(), a)
     with pytest.raises(ValueError, match="CUDA"):
         tg.gated_delta_scan(x, x, x, [0, 6], a, a)
+
+
+def test_topk_workspace_size_and_fused_gate_validation(L):
+    """The top-K workspace holds one 8448-byte block per prompt (2048 histogram
+    bins and a tag); the fused gate and the workspace selection refuse a
+    missing or short workspace and a batch that does not cover n_tokens,
+    before anything launches."""
+    assert L.tg_topk_workspace_bytes(1, 16384) == 8448
+    assert L.tg_topk_workspace_bytes(4, 147456) == 4 * 8448
+    assert L.tg_topk_workspace_bytes(0, 0) == 0
+    assert L.tg_topk_workspace_bytes(129, 0) == 0
+    _, cu_p = _arr([0, 100, 356])
+    _, s_p = _arr([0, 0])
+    _, e_p = _arr([90, 250])
+    _, k_p = _arr([10, 20])
+    gh = L.tg_gate_score_hist
+    args = (FAKE, 0, 356, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 2, cu_p, s_p, e_p)
+    assert gh(*args, None, 2 * 8448, 0, None) == INVALID        # no workspace
+    assert gh(*args, FAKE, 2 * 8448 - 1, 0, None) == WORKSPACE  # one byte short
+    assert gh(*args, FAKE_ODD, 2 * 8448, 0, None) == ALIGN
+    bad = (FAKE, 0, 355, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 2, cu_p, s_p, e_p)
+    assert gh(*bad, FAKE, 2 * 8448, 0, None) == SHAPE           # cu_seqlens ends at 356
+    _, e_bad = _arr([101, 250])
+    assert gh(FAKE, 0, 356, 64, FAKE, FAKE, 32, FAKE, 0.0, FAKE, 2, cu_p, s_p, e_bad, FAKE,
+              2 * 8448, 0, None) == INVALID                     # span past its prompt
+    ws = L.tg_topk_select_ws
+    assert ws(FAKE, 2, cu_p, s_p, e_p, k_p, FAKE, FAKE, None, 2 * 8448, None) == INVALID
+    assert ws(FAKE, 2, cu_p, s_p, e_p, k_p, FAKE, FAKE, FAKE, 8448, None) == WORKSPACE

@@ -6,8 +6,9 @@ import torch
 
 import learned_token_pruning_gate_b200 as tg
 from learned_token_pruning_gate_b200 import inputs as gen
-from tests.parity_utils import (ATTN_BF16, ATTN_FP32, GATE_ATOL, LSE_ATOL, assert_close, dev,
-                                host_f32, kept_set_agrees, sample_rows)
+from tests.parity_utils import (ATTN_BF16, ATTN_FP32, GATE_ATOL, LOGSIG_TOL, LSE_ATOL,
+                                assert_close, assert_rope_close, dev, host_f32, kept_set_agrees,
+                                sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -39,28 +40,17 @@ def _oracle_chain(oracle, inp, rows=None):
     return dict(z=z, kept=kept, cu_kept=cu_kept)
 
 
-def _oracle_tail(oracle, inp, kept, cu_kept, z32, rows):
-    """Compaction and attention of the oracle on a given kept set and given scores
-    (the GPU's): always well defined, so the attention is always compared."""
-    w = inp.w
-    q = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("q"), w.n_q_heads, w.head_dim,
-                           w.rope_theta)
-    k = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("k"), w.n_kv_heads, w.head_dim,
-                           w.rope_theta)
-    v = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("v"))
-    ls = oracle.logsig(kept, inp.cu_seqlens, inp.doc_begin, inp.doc_end, z32)
-    return oracle.gated_attention(q, k, v, cu_kept, ls, inp.gain.numpy(), inp.temp.numpy(),
-                                  rows=rows)
-
-
 def _check_chain(oracle, inp, g, rows=None, gate_rows=None):
     """Every stage of the GPU chain against the oracle:
       - gate scores within 1e-3 (all rows, or the sampled gate_rows);
       - the selection bit-exact against the oracle's top-K on the GPU's scores,
         and, when the oracle scored every row, within the 1e-3 band of its own;
-      - the planted needle kept;
-      - the attention output (and LSE) against the oracle's compaction and
-        attention over the GPU's kept set and scores, at the dtype's bar."""
+      - the planted needle kept wherever the budget can hold it;
+      - the compaction of the GPU's kept rows: residual and v bit-exact, q and
+        k within one storage ulp of the oracle's fp64 RoPE, log-gates 1e-6;
+      - the attention on the GPU's compacted rows at the stage bar (output
+        and LSE), and the output of the oracle's own fp64 compaction and
+        attention of the GPU's kept set at the dtype's bar."""
     w = inp.w
     z = g["z"].cpu().numpy()
     kept = g["kept_idx"].cpu().numpy()
@@ -79,16 +69,45 @@ def _check_chain(oracle, inp, g, rows=None, gate_rows=None):
                                           inp.budget)
     np.testing.assert_array_equal(kept, ref_kept)
     np.testing.assert_array_equal(cu_kept, ref_cu)
-    for rows_b in inp.needle_rows:  # the planted needle always survives
-        assert set(rows_b.tolist()) <= set(kept.tolist())
-    out_ref, lse_ref = _oracle_tail(oracle, inp, kept, cu_kept, z, rows)
+    for b, rows_b in enumerate(inp.needle_rows):  # the planted needle survives
+        if inp.budget[b] >= len(rows_b):
+            assert set(rows_b.tolist()) <= set(kept.tolist())
+    # compaction
+    kt = torch.from_numpy(kept.astype(np.int64))
+    for name in ("h", "v"):
+        np.testing.assert_array_equal(g[name].cpu().view(torch.int16 if w.dtype == "bf16"
+                                                         else torch.int32).numpy(),
+                                      getattr(inp, name)[kt].view(
+                                          torch.int16 if w.dtype == "bf16" else torch.int32
+                                      ).numpy())
+    ref_q = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("q"), w.n_q_heads, w.head_dim,
+                               w.rope_theta)
+    ref_k = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("k"), w.n_kv_heads, w.head_dim,
+                               w.rope_theta)
+    v64 = oracle.gather_rows(kept, inp.cu_seqlens, inp.f32("v"))
+    if w.dtype == "bf16":
+        assert_rope_close("q'", host_f32(g["q"]), ref_q)
+        assert_rope_close("k'", host_f32(g["k"]), ref_k)
+    else:
+        assert_close("q'", host_f32(g["q"]), ref_q, 1e-5, 1e-5)
+        assert_close("k'", host_f32(g["k"]), ref_k, 1e-5, 1e-5)
+    ls = oracle.logsig(kept, inp.cu_seqlens, inp.doc_begin, inp.doc_end, z)
+    assert_close("logsig", g["logsig"].cpu().numpy(), ls, *LOGSIG_TOL)
+    # attention on the GPU's compacted rows (the stage's own inputs)
+    tol = ATTN_FP32 if w.dtype == "fp32" else ATTN_BF16
     got = host_f32(g["out"])
     lse = g["lse"].cpu().numpy().T  # [M, Hq]
     if rows is not None:
         got, lse = got[rows], lse[rows]
-    tol = ATTN_FP32 if w.dtype == "fp32" else ATTN_BF16
-    assert_close("out", got, out_ref, *tol)
-    assert_close("lse", lse, lse_ref, LSE_ATOL, 0.0)
+    out_s, lse_s = oracle.gated_attention(host_f32(g["q"]), host_f32(g["k"]), host_f32(g["v"]),
+                                          cu_kept, g["logsig"].cpu().numpy(), inp.gain.numpy(),
+                                          inp.temp.numpy(), rows=rows)
+    assert_close("out (stage)", got, out_s, *tol)
+    assert_close("lse (stage)", lse, lse_s, LSE_ATOL, 1e-5)
+    # end to end: the oracle's fp64 compaction and attention of the same kept set
+    out_e, _ = oracle.gated_attention(ref_q, ref_k, v64, cu_kept, ls, inp.gain.numpy(),
+                                      inp.temp.numpy(), rows=rows)
+    assert_close("out (end to end)", got, out_e, *tol)
 
 
 @pytest.mark.parametrize("name,algo", [("tiny_fp32", tg.ALGO_AUTO), ("tiny_fp32", tg.ALGO_SIMT),

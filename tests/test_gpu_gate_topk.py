@@ -202,3 +202,111 @@ def test_topk_longest_prompt(oracle):
     z2 = torch.from_numpy(gen.random_scores(n + 1, seed=80)).cuda()
     with pytest.raises(tg.TokenGateError, match="TG_ERR_UNSUPPORTED.*exceeds"):
         tg.topk_select(z2, [0, n + 1], [0], [n], [1000])
+
+
+# ---- the selection's first radix pass counted by the gate ---------------------
+
+def _fused(inp, ws, algo=tg.ALGO_AUTO, z=None):
+    z = tg.gate_score(dev(inp.h), dev(inp.W1), dev(inp.b1), dev(inp.w2), inp.b2, out=z,
+                      algo=algo, topk_ws=ws, cu_seqlens=inp.cu_seqlens, doc_begin=inp.doc_begin,
+                      doc_end=inp.doc_end)
+    return z
+
+
+def _select_ws(oracle, inp, z, ws):
+    kept, cu_kept, host = tg.topk_select(z, inp.cu_seqlens, inp.doc_begin, inp.doc_end,
+                                         inp.budget, workspace=ws)
+    ref_kept, ref_cu = oracle.topk_select(z.cpu().numpy(), inp.cu_seqlens, inp.doc_begin,
+                                          inp.doc_end, inp.budget)
+    np.testing.assert_array_equal(kept.cpu().numpy(), ref_kept)
+    np.testing.assert_array_equal(cu_kept.cpu().numpy(), ref_cu)
+    torch.cuda.synchronize()
+    assert int(ws.count_nonzero()) == 0, "the selection must leave the workspace zeroed"
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "qwen_16k", "qwen_32k_k4096", "qwen_128k",
+                                  "ragged_4"])
+def test_fused_gate_selection_bit_exact(oracle, name):
+    """Gate with the first-pass histograms, then the selection from them: the
+    kept rows equal the oracle's top-K of the same scores, bit for bit, and the
+    scores equal the plain gate's exactly (the histogram changes no score)."""
+    w = gen.WORKLOADS[name]
+    inp = gen.make_inputs(w, with_qkv=False)
+    ws = tg.topk_workspace(w.batch)
+    z = _fused(inp, ws)
+    z_plain = tg.gate_score(dev(inp.h), dev(inp.W1), dev(inp.b1), dev(inp.w2), inp.b2)
+    assert torch.equal(z, z_plain)
+    _select_ws(oracle, inp, z, ws)
+
+
+def test_fused_histogram_counts_every_document_token(oracle):
+    """The gate's histogram of each prompt is exactly the count of its document
+    tokens' scores by the top 11 bits of the order key (read before any
+    selection consumes it), and the tag names the scores."""
+    w = gen.Workload("hist", (300, 0, 1000, 64, 2049), (20, 0, 1000, 3, 49), (5, 1, 10, 0, 100),
+                     256, 64, 4, 2, 64, "bf16", 4, 31)
+    inp = gen.make_inputs(w, with_qkv=False)
+    ws = tg.topk_workspace(w.batch)
+    z = _fused(inp, ws)
+    torch.cuda.synchronize()
+    words = ws.view(torch.int32).cpu().numpy().view(np.uint32).reshape(w.batch, 2112)
+    u = z.cpu().numpy().view(np.uint32).copy()
+    u[u == 0x80000000] = 0  # -0.0 counts as +0.0
+    key = np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+    key[np.isnan(z.cpu().numpy())] = 0
+    for b in range(w.batch):
+        s = inp.cu_seqlens[b] + inp.doc_begin[b]
+        e = inp.cu_seqlens[b] + inp.doc_end[b]
+        ref = np.bincount(key[s:e] >> 21, minlength=2048)
+        np.testing.assert_array_equal(words[b, :2048], ref)
+        assert words[b, 2048] == 0x7A6E5B1F and words[b, 2049] == w.total_tokens
+        assert (int(words[b, 2051]) << 32 | int(words[b, 2050])) == z.data_ptr()
+    # the selection consumes them and leaves the workspace zeroed
+    _select_ws(oracle, inp, z, ws)
+
+
+def test_fused_selection_falls_back_when_the_histogram_does_not_fit(oracle):
+    """The selection counts the first pass itself when the workspace does not
+    hold a histogram of these scores: never counted (zero), counted twice (two
+    gate calls, twice the tokens), or counted from scores at another address.
+    The kept rows are exact in every case and the workspace ends zeroed."""
+    w = gen.WORKLOADS["qwen_16k"]
+    inp = gen.make_inputs(w, with_qkv=False)
+    ws = tg.topk_workspace(w.batch)
+    z = _fused(inp, ws)
+    torch.cuda.synchronize()
+    ws.zero_()                                   # never counted
+    _select_ws(oracle, inp, z, ws)
+    _fused(inp, ws, z=z)
+    _fused(inp, ws, z=z)                         # counted twice
+    _select_ws(oracle, inp, z, ws)
+    other = torch.empty_like(z)
+    _fused(inp, ws, z=other)                     # the tag names `other`
+    _select_ws(oracle, inp, z.clone(), ws)
+
+
+def test_fused_selection_edge_batches(oracle):
+    """Empty prompts, K = 0, K >= n_doc, an all-question prompt, a document in
+    the middle, one-token prompts, and TG_MAX_BATCH prompts, through the
+    CUDA-core gate (fp32) and the tensor-core gate (bf16)."""
+    rng = np.random.default_rng(5)
+    B = tg.MAX_BATCH
+    seq = rng.integers(1, 600, size=B)
+    seq[::17] = 1
+    seq[5] = 0
+    qn = np.minimum(seq, rng.integers(0, 40, size=B))
+    bud = rng.integers(0, 300, size=B)
+    bud[::11] = 0
+    for dt, algo in (("bf16", tg.ALGO_AUTO), ("fp32", tg.ALGO_SIMT)):
+        w = gen.Workload("edges", tuple(int(x) for x in seq), tuple(int(x) for x in qn),
+                         tuple(int(x) for x in bud), 128, 32, 4, 2, 64, dt, 1, 17)
+        inp = gen.make_inputs(w, with_qkv=False)
+        ws = tg.topk_workspace(w.batch)
+        _select_ws(oracle, inp, _fused(inp, ws, algo), ws)
+    # a document span in the middle of its prompt (question before and after)
+    w = gen.Workload("mid", (5000, 3000), (0, 0), (700, 2999), 128, 32, 4, 2, 64, "bf16", 1, 18)
+    inp = gen.make_inputs(w, with_qkv=False)
+    inp.doc_begin[:] = [1000, 1]
+    inp.doc_end[:] = [4000, 3000]
+    ws = tg.topk_workspace(w.batch)
+    _select_ws(oracle, inp, _fused(inp, ws), ws)

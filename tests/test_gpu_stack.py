@@ -78,9 +78,12 @@ def test_stack_matches_oracle(lens, n_layers, dm, Hq, Hkv, dh, inter):
     assert tg.device_status() == 0
     lay = [{k: host_f32(v).astype(np.float64) for k, v in ly.items()} for ly in layers]
     rx, rk, rv = so.stack(host_f32(x0), pos, cu, ls.numpy(), lay, Hq, Hkv, dh)
+    # per element |gpu - ref| <= 2e-2 rms + 2e-2 |ref|: bf16 storage of every
+    # intermediate (x, the projections, q/k/v) and bf16 GEMM inputs put errors of
+    # a few bf16 units of the typical magnitude on every element, independent of
+    # the element's own size (measured need at rtol 2e-2: <= 1.3e-2 rms)
     for name, got, ref in [("x", x, rx), ("cache_k", ck, rk), ("cache_v", cv, rv)]:
         ref = np.asarray(ref, np.float64)
         g = host_f32(got).astype(np.float64).reshape(ref.shape)
         rms = np.sqrt(np.mean(ref * ref))
-        err = np.abs(g - ref).max() / rms
-        assert err <= 0.04, f"{name}: max error {err:.3e} of rms {rms:.3e}"
+        assert_close(name, g, ref, 2e-2 * rms, 2e-2)
