@@ -181,23 +181,38 @@ def _time_steps(graph, flush, stream, K, warmup, settle_s=0.3):
 
 
 def _time_stages(layer, flush, stream, n):
-    """Each of the step's launches alone, n times, one event pair each (ms, mean)."""
+    """Per-kernel times inside the step: the four launches captured in one CUDA
+    graph with an event record before and after each (on the launching stream),
+    replayed n times with an L2 flush between replays; a stage's time is the
+    interval between the events around its launch (mean over the replays).  The
+    records sit between the kernels, so the next launch cannot start early under
+    them: the sum of the stages is a little above the step time."""
     import ctypes
 
     import torch
 
-    kev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(n)] for s in layer.STAGES}
-    st = ctypes.c_void_p(stream.cuda_stream)
-    torch.cuda._sleep(HOLD_CYCLES)
-    for i in range(n):
-        flush.zero_()
-        for s in layer.STAGES:
-            kev[s][i][0].record(stream)
+    stages = layer.STAGES
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)]
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        st = ctypes.c_void_p(side.cuda_stream)
+        evs[0].record(side)
+        for j, s in enumerate(stages):
             getattr(layer, s)(st)
-            kev[s][i][1].record(stream)
+            evs[j + 1].record(side)
     torch.cuda.synchronize()
-    return {s: float(np.mean([a.elapsed_time(b) for a, b in kev[s]])) for s in kev}
+    acc = {s: [] for s in stages}
+    for i in range(n + 2):  # two untimed replays first
+        flush.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        if i >= 2:
+            for j, s in enumerate(stages):
+                acc[s].append(evs[j].elapsed_time(evs[j + 1]))
+    del g
+    return {s: float(np.mean(v)) for s, v in acc.items()}
 
 
 def _stages_and_roofline(tg, layer, w, name, stage_ms, pk):
@@ -516,7 +531,10 @@ def run_ncu_case(args):
         _, dq, dkk, dvv, dla, dbeta = gen.delta_inputs([layer.M], w.n_q_heads, w.head_dim, w.seed,
                                                        w.dtype)
         dq, dkk, dvv, dla, dbeta = (d(x) for x in (dq, dkk, dvv, dla, dbeta))
-        delta = lambda: tg.gated_delta_scan(dq, dkk, dvv, layer.cu_kept_host, dla, dbeta)  # noqa: E731
+        dws = torch.empty(tg.delta_scan_workspace_bytes(layer.cu_kept_host, w.n_q_heads, w.head_dim),
+                          dtype=torch.uint8, device="cuda")
+        delta = lambda: tg.gated_delta_scan(dq, dkk, dvv, layer.cu_kept_host, dla, dbeta,  # noqa: E731
+                                            algo=args.delta_algo, workspace=dws)
     for _ in range(args.steps):
         layer.run()
         if bwd:
@@ -641,17 +659,24 @@ def run_extras(args):
     d_out = torch.empty_like(dvv)
     d_state = torch.empty((len(dcu) - 1, w.n_q_heads, w.head_dim, w.head_dim), dtype=torch.float32,
                           device=dev)
+    rec_us = timed(lambda: tg.gated_delta_scan(dq, dkk, dvv, dcu, dla, dbeta, out=d_out,
+                                               state=d_state, algo="recurrent"), 10)
+    dws = torch.empty(tg.delta_scan_workspace_bytes(dcu, w.n_q_heads, w.head_dim), dtype=torch.uint8,
+                      device=dev)
     delta_us = timed(lambda: tg.gated_delta_scan(dq, dkk, dvv, dcu, dla, dbeta, out=d_out,
-                                                 state=d_state), 10)
-    # per row and head: S k, the rank-1 update (scale + FMA) and S q over d x d
+                                                 state=d_state, algo="chunked", workspace=dws), 10)
+    # per row and head, as the recurrence counts it: S k, the rank-1 update (scale
+    # + FMA) and S q over d x d -- the chunked form does about as many flops
     delta_flops = 7.0 * w.head_dim ** 2 * w.n_q_heads * Mk
-    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # FMA lanes x 2 flop x max SM clock, TFLOP/s
-    delta = {"us": round(delta_us, 2), "rows_per_s": round(Mk / delta_us * 1e6),
+    fp32_peak = FP32_FMA_TFLOPS
+    delta = {"us": round(delta_us, 2), "recurrent_us": round(rec_us, 2),
+             "rows_per_s": round(Mk / delta_us * 1e6),
              "tflops_fp32": round(delta_flops / delta_us / 1e6, 3),
              "frac_alu_nominal": round(delta_flops / delta_us / 1e6 / fp32_peak, 4),
-             "heads": w.n_q_heads, "head_dim": w.head_dim,
-             "note": "recurrent form: latency of one row's update chain x rows per prompt"}
-    del dq, dkk, dvv, dla, dbeta, d_out, d_state
+             "heads": w.n_q_heads, "head_dim": w.head_dim, "workspace_bytes": int(dws.numel()),
+             "note": "chunked scan (64-row chunks: parallel per-chunk solve, then the state "
+                     "passed chunk to chunk over 16-row blocks); recurrent_us: row by row"}
+    del dq, dkk, dvv, dla, dbeta, d_out, d_state, dws
     del layer, o_f, lse_f, dout, bws
     torch.cuda.synchronize()
     # ungated: every token of every prompt attends causally, no bias (the layer without a gate)
@@ -724,6 +749,8 @@ def main():
                     help="untimed: run --steps plain steps of the workload (profiling)")
     ap.add_argument("--delta", action="store_true",
                     help="with --ncu-case: also run the gated-delta-rule scan over the kept rows")
+    ap.add_argument("--delta-algo", default="chunked", choices=["chunked", "recurrent"],
+                    help="with --ncu-case --delta: which form of the scan")
     ap.add_argument("--backward", action="store_true",
                     help="with --ncu-case: also run the attention backward after each step")
     args = ap.parse_args()

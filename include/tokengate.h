@@ -228,6 +228,21 @@ TG_API tg_status tg_topk_select_multi(const float* z, int32_t batch, const int32
                                tg_stream_t stream);
 
 /*
+ * The budget sweep on a top-K workspace: the selections of tg_topk_select_multi
+ * (the same rows for every budget), with every budget's first radix pass taken
+ * from the one histogram tg_gate_score_hist counted from these scores -- the
+ * scores' histogram is computed once and each budget takes its threshold from
+ * it -- and the workspace left zeroed once the last budget has read it.
+ * Arguments as tg_topk_select_multi plus the workspace of tg_topk_select_ws.
+ */
+TG_API tg_status tg_topk_select_multi_ws(const float* z, int32_t batch,
+                                         const int32_t* cu_seqlens_h, const int32_t* doc_begin_h,
+                                         const int32_t* doc_end_h, int32_t n_budgets,
+                                         const int32_t* budgets_h, int32_t* const* kept_idx_out,
+                                         int32_t* const* cu_kept_out, void* workspace,
+                                         size_t workspace_bytes, tg_stream_t stream);
+
+/*
  * Random-K selection (pages: the random-K selector ablation, which keeps K
  * document tokens at random instead of by gate score).  The random numbers are
  * the caller's: keys[total_tokens] uint32, one per token (for example i.i.d.
@@ -467,6 +482,39 @@ TG_API tg_status tg_gated_delta_scan(const void* q, const void* k, const void* v
                                      const float* log_alpha, const float* beta, int32_t batch,
                                      const int32_t* cu_kept_h, int32_t n_heads, int32_t head_dim,
                                      float eps, void* out, float* state_out, tg_stream_t stream);
+
+/*
+ * tg_gated_delta_scan_chunked: the function of tg_gated_delta_scan (same
+ * arguments, results and errors, same tolerance to fp32 rounding) computed in
+ * chunks of 64 rows.  With S_0 the state before a chunk, everything inside the
+ * chunk that does not involve S_0 -- the unit lower-triangular solve of the
+ * chunk's delta-rule corrections, the within-chunk decayed products of q, k and
+ * v -- is computed for every (chunk, head) at once, in parallel; the state then
+ * passes from chunk to chunk with three small products per chunk, split over
+ * blocks of 16 state rows (rows of S are independent).  This is the chunked
+ * linear-attention scan; the recurrence walks the rows one by one.
+ *   workspace  device scratch of tg_delta_scan_workspace_bytes bytes, 256-byte
+ *              aligned (TG_ERR_WORKSPACE when smaller or NULL with rows to scan,
+ *              TG_ERR_ALIGNMENT when misaligned); every call overwrites it, so
+ *              calls that share it must not overlap on the GPU.
+ *   batch x n_heads above 65535: TG_ERR_UNSUPPORTED.
+ */
+TG_API tg_status tg_gated_delta_scan_chunked(const void* q, const void* k, const void* v,
+                                             tg_dtype dtype, const float* log_alpha,
+                                             const float* beta, int32_t batch,
+                                             const int32_t* cu_kept_h, int32_t n_heads,
+                                             int32_t head_dim, float eps, void* out,
+                                             float* state_out, void* workspace,
+                                             size_t workspace_bytes, tg_stream_t stream);
+
+/*
+ * Workspace bytes tg_gated_delta_scan_chunked needs (host-only): per chunk of 64
+ * kept rows of a prompt and per head, five 64 x head_dim fp32 matrices and the
+ * chunk's decay (about 160 KB at head_dim 128).
+ */
+TG_API tg_status tg_delta_scan_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,
+                                               int32_t n_heads, int32_t head_dim,
+                                               size_t* bytes_out);
 
 /* Workspace bytes tg_gated_attention_backward needs for this batch (host-only). */
 TG_API tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,

@@ -26,7 +26,7 @@ __all__ = [
     "gated_prefill", "device_status", "EXPORTED_SYMBOLS", "attention_workspace_bytes",
     "attention_kernel", "topk_select_multi", "random_select", "gated_attention_backward",
     "attention_backward_workspace_bytes", "rmsnorm", "qkv_rope_emit", "swiglu", "gated_delta_scan",
-    "topk_workspace_bytes", "topk_workspace",
+    "topk_workspace_bytes", "topk_workspace", "delta_scan_workspace_bytes",
 ]
 
 TG_BF16, TG_FP32 = 0, 1
@@ -45,6 +45,7 @@ EXPORTED_SYMBOLS = (
     "tg_gated_attention_backward", "tg_attention_backward_workspace_bytes", "tg_rmsnorm",
     "tg_qkv_rope_emit", "tg_swiglu", "tg_gated_delta_scan", "tg_last_device_error",
     "tg_topk_workspace_bytes", "tg_gate_score_hist", "tg_topk_select_ws",
+    "tg_gated_delta_scan_chunked", "tg_delta_scan_workspace_bytes", "tg_topk_select_multi_ws",
 )
 MAX_BUDGETS = 8
 ATTN_KERNELS = {0: "attn_simt_kernel", 1: "attn_tc_kernel", 2: "attn_tc_kernel (key-range split)",
@@ -96,6 +97,9 @@ def library():
                                     ctypes.c_size_t, _vp]
     L.tg_topk_select_multi.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32, _i32p,
                                        ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp]
+    L.tg_topk_select_multi_ws.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32, _i32p,
+                                          ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp,
+                                          ctypes.c_size_t, _vp]
     L.tg_random_select.argtypes = [_vp, _i32, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp]
     L.tg_compact_gather.argtypes = [_vp, _i64, _i32, _i32p, _i32p, _i32p, _i32p, ctypes.c_int,
                                     ctypes.POINTER(GatherTensor), _i32, _i32, ctypes.c_double,
@@ -119,6 +123,11 @@ def library():
     L.tg_swiglu.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i32, _vp]
     L.tg_gated_delta_scan.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _i32, _i32p, _i32, _i32,
                                       _f32, _vp, _vp, _vp]
+    L.tg_gated_delta_scan_chunked.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _i32, _i32p,
+                                              _i32, _i32, _f32, _vp, _vp, _vp, ctypes.c_size_t,
+                                              _vp]
+    L.tg_delta_scan_workspace_bytes.argtypes = [_i32, _i32p, _i32, _i32,
+                                                ctypes.POINTER(ctypes.c_size_t)]
     for name in EXPORTED_SYMBOLS:
         if name not in ("tg_status_string", "tg_last_error_message", "tg_version",
                         "tg_topk_workspace_bytes"):
@@ -281,9 +290,11 @@ def topk_select(z, cu_seqlens, doc_begin, doc_end, budget, kept_idx=None, cu_kep
     return kept_idx, cu_kept, host
 
 
-def topk_select_multi(z, cu_seqlens, doc_begin, doc_end, budgets):
+def topk_select_multi(z, cu_seqlens, doc_begin, doc_end, budgets, workspace=None):
     """Top-K for a budget sweep from one score vector: budgets is a list of
-    per-prompt budget lists (at most MAX_BUDGETS).  One launch.
+    per-prompt budget lists (at most MAX_BUDGETS).  One launch.  With
+    ``workspace`` (a top-K workspace the gate counted these scores into, see
+    gate_score) every budget takes its first radix pass from that one histogram.
 
     Returns a list of (kept_idx [M_q] device, cu_kept [B+1] device, cu_kept_host).
     """
@@ -301,9 +312,17 @@ def topk_select_multi(z, cu_seqlens, doc_begin, doc_end, budgets):
         cuk = torch.empty(len(s) + 1, dtype=torch.int32, device=z.device)
         kept_ptrs[q], cu_ptrs[q] = kept.data_ptr() if M else None, cuk.data_ptr()
         outs.append((kept, cuk, host))
-    _check("tg_topk_select_multi", library().tg_topk_select_multi(
+    if workspace is None:
+        _check("tg_topk_select_multi", library().tg_topk_select_multi(
+            _ptr(z), len(s), cu_p, s_p, e_p, len(ks), ks.ctypes.data_as(_i32p), kept_ptrs,
+            cu_ptrs, _stream(z.device)))
+        return outs
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or \
+            workspace.device != z.device:
+        raise ValueError("workspace must be a contiguous uint8 tensor on z's device")
+    _check("tg_topk_select_multi_ws", library().tg_topk_select_multi_ws(
         _ptr(z), len(s), cu_p, s_p, e_p, len(ks), ks.ctypes.data_as(_i32p), kept_ptrs, cu_ptrs,
-        _stream(z.device)))
+        _ptr(workspace), workspace.numel(), _stream(z.device)))
     return outs
 
 
@@ -559,11 +578,26 @@ def swiglu(gate_up, out=None):
     return out
 
 
+def delta_scan_workspace_bytes(cu_kept_host, n_heads, head_dim):
+    """Device scratch bytes the chunked delta-rule scan needs for this batch."""
+    ck, ck_p = _host_i32(cu_kept_host)
+    out = ctypes.c_size_t(0)
+    _check("tg_delta_scan_workspace_bytes", library().tg_delta_scan_workspace_bytes(
+        len(ck) - 1, ck_p, int(n_heads), int(head_dim), ctypes.byref(out)))
+    return int(out.value)
+
+
 def gated_delta_scan(q, k, v, cu_kept_host, log_alpha, beta, eps=1e-6, out=None, state=None,
-                     want_state=True):
+                     want_state=True, algo="chunked", workspace=None):
     """Gated delta rule over each prompt's kept rows (a Gated DeltaNet layer above the
     gate): q, k, v [M, H, d] (d 64 or 128), log_alpha, beta [M, H] fp32.  Returns
-    (o [M, H, d], state [B, H, d, d] fp32 or None)."""
+    (o [M, H, d], state [B, H, d, d] fp32 or None).
+
+    algo: "chunked" (tg_gated_delta_scan_chunked: parallel within chunks of 64
+    rows; ``workspace`` a uint8 device tensor of delta_scan_workspace_bytes, or
+    None to allocate one) or "recurrent" (tg_gated_delta_scan: row by row)."""
+    if algo not in ("chunked", "recurrent"):
+        raise ValueError(f"algo {algo!r}: 'chunked' or 'recurrent'")
     if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
         raise ValueError(f"q, k, v must share one [M, H, d] shape: {tuple(q.shape)}, "
                          f"{tuple(k.shape)}, {tuple(v.shape)}")
@@ -587,9 +621,22 @@ def gated_delta_scan(q, k, v, cu_kept_host, log_alpha, beta, eps=1e-6, out=None,
         out = torch.empty_like(v)
     if state is None and want_state:
         state = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
-    _check("tg_gated_delta_scan", library().tg_gated_delta_scan(
+    if algo == "recurrent":
+        _check("tg_gated_delta_scan", library().tg_gated_delta_scan(
+            _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), B, ck_p, H, d,
+            float(eps), _ptr(out), _ptr(state) if state is not None else None,
+            _stream(q.device)))
+        return out, state
+    if workspace is None:
+        nbytes = delta_scan_workspace_bytes(ck, H, d)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    elif workspace.dtype != torch.uint8 or not workspace.is_contiguous() or \
+            workspace.device != q.device:
+        raise ValueError("workspace must be a contiguous uint8 tensor on q's device")
+    _check("tg_gated_delta_scan_chunked", library().tg_gated_delta_scan_chunked(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), B, ck_p, H, d,
-        float(eps), _ptr(out), _ptr(state) if state is not None else None, _stream(q.device)))
+        float(eps), _ptr(out), _ptr(state) if state is not None else None, _ptr(workspace),
+        workspace.numel(), _stream(q.device)))
     return out, state
 
 

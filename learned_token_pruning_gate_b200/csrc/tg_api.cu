@@ -371,11 +371,42 @@ tg_status tg_topk_select_ws(const float* z, int32_t batch, const int32_t* cu_seq
                           cu_kept_out, static_cast<uint32_t*>(workspace), stream);
 }
 
+static tg_status topk_select_multi_impl(const float* z, int32_t batch,
+                                        const int32_t* cu_seqlens_h, const int32_t* doc_begin_h,
+                                        const int32_t* doc_end_h, int32_t n_budgets,
+                                        const int32_t* budgets_h, int32_t* const* kept_idx_out,
+                                        int32_t* const* cu_kept_out, uint32_t* hist,
+                                        tg_stream_t stream);
+
 tg_status tg_topk_select_multi(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
                                const int32_t* doc_begin_h, const int32_t* doc_end_h,
                                int32_t n_budgets, const int32_t* budgets_h,
                                int32_t* const* kept_idx_out, int32_t* const* cu_kept_out,
                                tg_stream_t stream) {
+  return topk_select_multi_impl(z, batch, cu_seqlens_h, doc_begin_h, doc_end_h, n_budgets,
+                                budgets_h, kept_idx_out, cu_kept_out, nullptr, stream);
+}
+
+tg_status tg_topk_select_multi_ws(const float* z, int32_t batch, const int32_t* cu_seqlens_h,
+                                  const int32_t* doc_begin_h, const int32_t* doc_end_h,
+                                  int32_t n_budgets, const int32_t* budgets_h,
+                                  int32_t* const* kept_idx_out, int32_t* const* cu_kept_out,
+                                  void* workspace, size_t workspace_bytes, tg_stream_t stream) {
+  if (batch > 0 && batch <= kMaxBatch) {
+    tg_status r = check_topk_workspace(batch, workspace, workspace_bytes);
+    if (r != TG_OK) return r;
+  }
+  return topk_select_multi_impl(z, batch, cu_seqlens_h, doc_begin_h, doc_end_h, n_budgets,
+                                budgets_h, kept_idx_out, cu_kept_out,
+                                static_cast<uint32_t*>(workspace), stream);
+}
+
+static tg_status topk_select_multi_impl(const float* z, int32_t batch,
+                                        const int32_t* cu_seqlens_h, const int32_t* doc_begin_h,
+                                        const int32_t* doc_end_h, int32_t n_budgets,
+                                        const int32_t* budgets_h, int32_t* const* kept_idx_out,
+                                        int32_t* const* cu_kept_out, uint32_t* hist,
+                                        tg_stream_t stream) {
   if (n_budgets < 1 || n_budgets > TG_MAX_BUDGETS)
     return set_error(TG_ERR_INVALID_ARG, "n_budgets=%d (1..%d)", n_budgets, TG_MAX_BUDGETS);
   if (!budgets_h || !kept_idx_out) return set_error(TG_ERR_INVALID_ARG, "null budget array");
@@ -393,7 +424,7 @@ tg_status tg_topk_select_multi(const float* z, int32_t batch, const int32_t* cu_
   if (t[0].start[batch] > 0 && !z) return set_error(TG_ERR_INVALID_ARG, "z is null");
   if (max_len > 360448)
     return set_error(TG_ERR_UNSUPPORTED, "prompt of %d tokens exceeds 360448", max_len);
-  return launch_topk(z, nullptr, t, n_budgets, max_len, kept_idx_out, cu_kept_out, nullptr,
+  return launch_topk(z, nullptr, t, n_budgets, max_len, kept_idx_out, cu_kept_out, hist,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -616,6 +647,64 @@ tg_status tg_gated_delta_scan(const void* q, const void* k, const void* v, tg_dt
       return set_error(TG_ERR_ALIGNMENT, "q, k, v and state_out must be 16-byte aligned");
   return launch_delta_scan(q, k, v, dtype, log_alpha, beta, t, n_heads, head_dim, eps, out, state_out,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Shared argument checks of the two forms of the delta-rule scan.
+static tg_status check_delta_args(const void* q, const void* k, const void* v, tg_dtype dtype,
+                                  const float* log_alpha, const float* beta, int32_t batch,
+                                  const int32_t* cu_kept_h, int32_t n_heads, int32_t head_dim,
+                                  float eps, void* out, float* state_out, PromptTable* t) {
+  if (dtype != TG_BF16 && dtype != TG_FP32) return set_error(TG_ERR_DTYPE, "dtype %d", dtype);
+  int max_len = 0;
+  tg_status r = build_kept_table(batch, cu_kept_h, t, &max_len);
+  if (r != TG_OK) return r;
+  if (n_heads <= 0) return set_error(TG_ERR_SHAPE, "n_heads=%d", n_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(TG_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", head_dim);
+  if (!(eps >= 0.0f)) return set_error(TG_ERR_INVALID_ARG, "eps must be >= 0");
+  if (t->kept_start[batch] > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+    return set_error(TG_ERR_INVALID_ARG, "null pointer");
+  for (const void* ptr : {q, k, v, static_cast<const void*>(state_out)})
+    if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0)
+      return set_error(TG_ERR_ALIGNMENT, "q, k, v and state_out must be 16-byte aligned");
+  return TG_OK;
+}
+
+tg_status tg_delta_scan_workspace_bytes(int32_t batch, const int32_t* cu_kept_h, int32_t n_heads,
+                                        int32_t head_dim, size_t* bytes_out) {
+  if (!bytes_out) return set_error(TG_ERR_INVALID_ARG, "bytes_out is NULL");
+  *bytes_out = 0;
+  PromptTable t;
+  int max_len = 0;
+  tg_status r = build_kept_table(batch, cu_kept_h, &t, &max_len);
+  if (r != TG_OK) return r;
+  if (n_heads <= 0) return set_error(TG_ERR_SHAPE, "n_heads=%d", n_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(TG_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", head_dim);
+  *bytes_out = delta_chunked_workspace_bytes(t, n_heads, head_dim);
+  return TG_OK;
+}
+
+tg_status tg_gated_delta_scan_chunked(const void* q, const void* k, const void* v, tg_dtype dtype,
+                                      const float* log_alpha, const float* beta, int32_t batch,
+                                      const int32_t* cu_kept_h, int32_t n_heads, int32_t head_dim,
+                                      float eps, void* out, float* state_out, void* workspace,
+                                      size_t workspace_bytes, tg_stream_t stream) {
+  PromptTable t;
+  tg_status r = check_delta_args(q, k, v, dtype, log_alpha, beta, batch, cu_kept_h, n_heads,
+                                 head_dim, eps, out, state_out, &t);
+  if (r != TG_OK) return r;
+  if (static_cast<int64_t>(batch) * n_heads > 65535)
+    return set_error(TG_ERR_UNSUPPORTED, "n_heads=%d exceeds one launch", n_heads);
+  if (batch == 0 || (t.kept_start[batch] == 0 && !state_out)) return TG_OK;
+  const size_t need = delta_chunked_workspace_bytes(t, n_heads, head_dim);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return set_error(TG_ERR_WORKSPACE, "delta-scan workspace: %zu bytes given, %zu needed",
+                     workspace ? workspace_bytes : 0, need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+    return set_error(TG_ERR_ALIGNMENT, "the delta-scan workspace must be 256-byte aligned");
+  return launch_delta_chunked(q, k, v, dtype, log_alpha, beta, t, n_heads, head_dim, eps, out,
+                              state_out, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 tg_status tg_attention_backward_workspace_bytes(int32_t batch, const int32_t* cu_kept_h,

@@ -424,6 +424,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = tmem + lane_off + 256 + x * 128;
     uint32_t s_waits = 0, o_waits = 0, tile_ctr = 0;
     bool ok = true;
+    // A unit's output is packed in registers and stored only after the next
+    // unit's bias operands are published: a release arrival waits for the
+    // thread's earlier global stores, and the O-free and bias arrivals gate the
+    // tensor core, so the stores must not precede them.
+    uint32_t pend[DH / 32][16];
+    uint4* pend_dst = nullptr;
+    float* pend_lse = nullptr;
+    float pend_lse_v = 0.0f;
+    auto flush = [&]() {
+      if (pend_dst) {
+#pragma unroll
+        for (int c = 0; c < DH / 32; ++c)
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            pend_dst[c * 4 + v4] = make_uint4(pend[c][4 * v4], pend[c][4 * v4 + 1],
+                                              pend[c][4 * v4 + 2], pend[c][4 * v4 + 3]);
+        pend_dst = nullptr;
+      }
+      if (pend_lse) {
+        *pend_lse = pend_lse_v;
+        pend_lse = nullptr;
+      }
+    };
     for (int round = 0; ok; ++round) {
       const int u = snake_unit(round, blockIdx.x, gridDim.x);
       if (u >= p.n_units) break;
@@ -474,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(kAugFull + x));
+      flush();  // the previous unit's output, now that its successor may start
       float m = -INFINITY, l = 0.0f;
       for (int j = 0; j < n_kv; ++j) {
         const int jabs = w.j0 + j;
@@ -591,24 +615,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t orow[32];
           tmem_ld32(t_o + c * 32, orow);
           tmem_ld_wait(orow);
-          if (qi < len) {
-            uint32_t pkd[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(orow[2 * e]) * inv,
-                                                        __uint_as_float(orow[2 * e + 1]) * inv);
-              pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(orow[2 * e]) * inv,
+                                                      __uint_as_float(orow[2 * e + 1]) * inv);
+            pend[c][e] = *reinterpret_cast<uint32_t*>(&pp);
           }
         }
         tc_fence_before();
         mbar_arrive(bar(kOFree + x));
-        if (p.lse && qi < len)
-          p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (m + log2f(l)) * kLn2;
+        if (qi < len) pend_dst = reinterpret_cast<uint4*>(out);
+        if (p.lse && qi < len) {
+          pend_lse = p.lse + static_cast<int64_t>(head) * p.m_total + kstart + qi;
+          pend_lse_v = (m + log2f(l)) * kLn2;
+        }
       } else {
         // chunk of a split item: store the normalised partial and its log2 LSE
         constexpr int kV4 = DH / 4;
@@ -720,6 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(kOFree + x));  // O may now be overwritten by the next unit
       }
     }
+    flush();
   }
 
   tc_fence_before();
@@ -1040,6 +1061,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const uint32_t t_o = tmem + lane_off + 256 + wg * 128;
     uint32_t s_ph = 0, o_waits = 0;
     bool ok = true;
+    // The output of a unit is packed in registers and stored only after the next
+    // unit's bias operands are published: a release arrival waits for the
+    // thread's earlier global stores, and the O-free and bias arrivals gate the
+    // tensor core, so the stores must not precede them.
+    uint32_t pend[2][16];
+    uint4* pend_dst = nullptr;  // this thread's output row (columns of its warpgroup), or null
+    float* pend_lse = nullptr;
+    float pend_lse_v = 0.0f;
+    auto flush = [&]() {
+      if (pend_dst) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            pend_dst[cc * 4 + v4] = make_uint4(pend[cc][4 * v4], pend[cc][4 * v4 + 1],
+                                               pend[cc][4 * v4 + 2], pend[cc][4 * v4 + 3]);
+        pend_dst = nullptr;
+      }
+      if (pend_lse) {
+        *pend_lse = pend_lse_v;
+        pend_lse = nullptr;
+      }
+    };
     for (int round = 0; ok; ++round) {
       const int u = snake_unit(round, cl, ncl);
       if (u >= p.n_units) break;
@@ -1079,6 +1123,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       if (wg + 2 < n_kv) next_l = load_l(wg + 2);
       fence_proxy_async_smem();
       mbar_arrive_cluster(leader_bar(kPAugFull));
+      flush();  // the previous unit's output, now that its successor may start
       float m = -INFINITY, l = 0.0f;
       for (int j = wg; j < n_kv; j += 2) {
         const int jabs = w.j0 + j;
@@ -1206,29 +1251,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) o1[e] = 0u;
         }
-        if (qi < len) {
-          uint32_t pkd[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float v0 = two ? fmaf(__uint_as_float(o0[2 * e]), g0, __uint_as_float(o1[2 * e]) * g1)
-                                 : __uint_as_float(o0[2 * e]) * g0;
-            const float v1 = two ? fmaf(__uint_as_float(o0[2 * e + 1]), g0,
-                                        __uint_as_float(o1[2 * e + 1]) * g1)
-                                 : __uint_as_float(o0[2 * e + 1]) * g0;
-            __nv_bfloat162 pp = __floats2bfloat162_rn(v0, v1);
-            pkd[e] = *reinterpret_cast<uint32_t*>(&pp);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+        for (int e = 0; e < 16; ++e) {
+          const float v0 = two ? fmaf(__uint_as_float(o0[2 * e]), g0, __uint_as_float(o1[2 * e]) * g1)
+                               : __uint_as_float(o0[2 * e]) * g0;
+          const float v1 = two ? fmaf(__uint_as_float(o0[2 * e + 1]), g0,
+                                      __uint_as_float(o1[2 * e + 1]) * g1)
+                               : __uint_as_float(o0[2 * e + 1]) * g0;
+          __nv_bfloat162 pp = __floats2bfloat162_rn(v0, v1);
+          pend[cc][e] = *reinterpret_cast<uint32_t*>(&pp);
         }
       }
       tc_fence_before();
       mbar_arrive_cluster(leader_bar(kPOFree));
-      if (wg == 0 && p.lse && qi < len)
-        p.lse[static_cast<int64_t>(head) * p.m_total + kstart + qi] = (mm + log2f(lsum)) * kLn2;
+      if (qi < len) pend_dst = reinterpret_cast<uint4*>(out + wg * 64);
+      if (wg == 0 && p.lse && qi < len) {
+        pend_lse = p.lse + static_cast<int64_t>(head) * p.m_total + kstart + qi;
+        pend_lse_v = (mm + log2f(lsum)) * kLn2;
+      }
     }
+    flush();
     }
   }
 

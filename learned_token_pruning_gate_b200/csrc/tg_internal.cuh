@@ -29,8 +29,9 @@ struct PromptTable {
 
 // First-pass radix histograms handed from the gate to the top-K select (the
 // top-K workspace).  Per prompt: kHistBins counts of the top 11 bits of the
-// order key (below) of its document tokens' scores, then a 4-word tag {magic,
-// total tokens, score pointer lo, hi} naming the scores they were counted from.
+// order key (below) of its document tokens' scores, then a tag {magic, total
+// tokens, score pointer lo, hi} naming the scores they were counted from, and a
+// counter of the selections that have read them (word 4).
 constexpr int kHistBins = 2048;
 constexpr int kHistStride = 2112;  // words per prompt: 8448 bytes, a multiple of 256
 constexpr uint32_t kHistMagic = 0x7A6E5B1Fu;
@@ -119,6 +120,12 @@ tg_status launch_delta_scan(const void* q, const void* k, const void* v, tg_dtyp
                             int head_dim, float eps, void* out, float* state, cudaStream_t st);
 tg_status launch_swiglu(const void* gu, void* h, tg_dtype dt, int64_t rows, int inter,
                         cudaStream_t st);
+// Chunked form of the gated delta rule (workspace of delta_chunked_workspace_bytes).
+size_t delta_chunked_workspace_bytes(const PromptTable& pt, int heads, int head_dim);
+tg_status launch_delta_chunked(const void* q, const void* k, const void* v, tg_dtype dt,
+                               const float* log_alpha, const float* beta, const PromptTable& pt,
+                               int heads, int head_dim, float eps, void* out, float* state,
+                               void* workspace, cudaStream_t st);
 // Workspace the tensor-core attention uses to split long items on this device (0 = none).
 size_t attn_tc_workspace_bytes(const PromptTable& pt, int hq, int hkv, int dh);
 // The tg_attn_kernel the tensor-core attention launches for this batch.

@@ -16,7 +16,9 @@
 //     bits; usually the last pass is skipped for continuous scores).
 //     The first pass's histogram comes from the gate when it counted these
 //     scores into the top-K workspace (tg_gate_score_hist): every CTA reads
-//     the prompt's 2048 bins and picks the digit itself, with no exchange.
+//     the prompt's 2048 bins and picks the digit itself, with no exchange;
+//     in a budget sweep every budget takes its first digit from that one
+//     histogram.
 //     Otherwise, and for the later passes, each CTA adds its non-zero bins
 //     into every CTA's totals with remote shared-memory atomics, one cluster
 //     barrier publishes them, and every CTA scans its own copy, so all of them
@@ -52,6 +54,7 @@ struct TopkParams {
   const uint32_t* keys;  // caller keys (kKeys = true)
   uint32_t* status;
   uint32_t* hist;      // top-K workspace with the gate's first-pass histograms, or null
+  int32_t n_budgets;   // clusters per prompt that read the same histogram
   int32_t cluster;     // CTAs per (budget, prompt)
 };
 
@@ -302,11 +305,19 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const __grid_constant
     p.cu_kept[q][b + 1] = p.kept_start[q][b + 1];
     if (b == 0) p.cu_kept[q][0] = 0;
   }
-  // leave the workspace zeroed for the next gate (every CTA read it before the
-  // barriers above); the tag is cleared so the bins are never reused
+  // Leave the workspace zeroed for the next gate: every CTA of this cluster read
+  // it before the barriers above; the last of the prompt's budget clusters to
+  // get here (a counter in the tag) clears the bins and the tag, so they are
+  // never reused.
   if (hist_b && r == 0) {
-    for (int i = tid; i < kBins; i += kThreads) hist_b[i] = 0;
-    if (tid == 0) hist_b[kBins] = 0;
+    __shared__ uint32_t s_last;
+    if (tid == 0)
+      s_last = atomicAdd(hist_b + kBins + 4, 1u) == static_cast<uint32_t>(p.n_budgets - 1);
+    __syncthreads();
+    if (s_last) {
+      for (int i = tid; i < kBins; i += kThreads) hist_b[i] = 0;
+      if (tid < 8) hist_b[kBins + tid] = 0;
+    }
   }
 }
 
@@ -326,7 +337,8 @@ tg_status launch_topk(const float* z, const uint32_t* keys, const PromptTable* t
   }
   p.z = z;
   p.keys = keys;
-  p.hist = (n_budgets == 1 && !keys) ? hist : nullptr;
+  p.hist = keys ? nullptr : hist;
+  p.n_budgets = n_budgets;
   p.status = device_status_word();
   if (!p.status) return set_error(TG_ERR_CUDA, "device status word unavailable");
   const int cl = kMaxCluster;  // latency-bound: spread every prompt over 8 SMs

@@ -310,3 +310,28 @@ def test_fused_selection_edge_batches(oracle):
     inp.doc_end[:] = [4000, 3000]
     ws = tg.topk_workspace(w.batch)
     _select_ws(oracle, inp, _fused(inp, ws), ws)
+
+
+@pytest.mark.parametrize("name", ["qwen_16k", "ragged_4"])
+def test_fused_budget_sweep_shares_the_gate_histogram(oracle, name):
+    """A budget sweep on the gate's first-pass histogram: every budget's kept
+    rows equal the oracle's top-K of the same scores with that budget, and the
+    workspace is zero once the last budget has read it (budgets of 0, 1, the
+    whole document and in between, per prompt)."""
+    w = gen.WORKLOADS[name]
+    inp = gen.make_inputs(w, with_qkv=False)
+    n_doc = np.asarray(inp.doc_end) - np.asarray(inp.doc_begin)
+    sweep = [[0] * w.batch, [1] * w.batch, [int(x) for x in n_doc], [int(x) + 5 for x in n_doc]]
+    sweep += [[max(1, int(f * nd)) for nd in n_doc] for f in (0.03, 0.125, 0.5, 0.9)]
+    ws = tg.topk_workspace(w.batch)
+    z = _fused(inp, ws)
+    outs = tg.topk_select_multi(z, inp.cu_seqlens, inp.doc_begin, inp.doc_end, sweep,
+                                workspace=ws)
+    zh = z.cpu().numpy()
+    for (kept, cu_kept, host), bud in zip(outs, sweep):
+        ref_kept, ref_cu = oracle.topk_select(zh, inp.cu_seqlens, inp.doc_begin, inp.doc_end,
+                                              np.asarray(bud, np.int32))
+        np.testing.assert_array_equal(kept.cpu().numpy(), ref_kept)
+        np.testing.assert_array_equal(cu_kept.cpu().numpy(), ref_cu)
+    torch.cuda.synchronize()
+    assert int(ws.count_nonzero()) == 0
