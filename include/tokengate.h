@@ -106,7 +106,8 @@ TG_API tg_status tg_device_status(tg_stream_t stream, uint32_t* bits_out);
  * code_out.  Bits: 1 a gate pipeline wait gave up, 2 an attention wait gave
  * up (forward or backward), 4 the top-K selection produced more rows than M_b (extra rows skipped),
  * 8 a kept index outside the prompt batch reached the gather (row skipped),
- * 16 a gather pipeline wait gave up.
+ * 16 a gather pipeline wait gave up, 32 a chunk load of the chunked delta-rule
+ * scan did not land.
  */
 TG_API tg_status tg_last_device_error(tg_stream_t stream, int32_t* code_out);
 

@@ -54,6 +54,7 @@ enum : uint32_t {
   kDevTopkOverflow = 1u << 2,   // selection produced more rows than M_b (skipped)
   kDevGatherIndex = 1u << 3,    // a kept index outside the prompt batch (row skipped)
   kDevTimeoutGather = 1u << 4,
+  kDevTimeoutDelta = 1u << 5,   // a chunk load of the chunked delta-rule scan did not land
 };
 
 // Host side: error reporting and the device status word.
