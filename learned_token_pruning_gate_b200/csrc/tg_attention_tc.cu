@@ -1062,9 +1062,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     uint32_t s_ph = 0, o_waits = 0;
     bool ok = true;
     // The output of a unit is packed in registers and stored only after the next
-    // unit's bias operands are published: a release arrival waits for the
-    // thread's earlier global stores, and the O-free and bias arrivals gate the
-    // tensor core, so the stores must not precede them.
+    // unit's bias operands are published, so no store of this thread is still
+    // outstanding when it makes the O-free and bias arrivals that gate the
+    // tensor core.
     uint32_t pend[2][16];
     uint4* pend_dst = nullptr;  // this thread's output row (columns of its warpgroup), or null
     float* pend_lse = nullptr;

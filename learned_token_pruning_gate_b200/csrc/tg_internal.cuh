@@ -457,9 +457,15 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
 }
+// Arrival on a barrier that may live in the peer CTA of the pair.  Every use
+// hands the tensor core of the pair something this thread produced on its own
+// SM -- TMEM columns (ordered by tcgen05.wait and the tcgen05 fences) or
+// shared-memory operands (ordered by fence.proxy.async) -- so the arrival keeps
+// the default CTA-scope release.  A cluster-scope release also waits for the
+// thread's outstanding global memory operations (prefetch loads, output
+// stores), which put about half a microsecond on the softmax critical path.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // TMA load whose completion is counted on a barrier that may live in the peer CTA
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t x,
