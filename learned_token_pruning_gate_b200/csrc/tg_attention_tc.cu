@@ -794,7 +794,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 //              warpgroups merge O_0 and O_1, each for half of the columns.
 // ---------------------------------------------------------------------------
 constexpr int kPairThreads = 384;
-constexpr int kPKStages = 5, kPVStages = 5;
+// Three stages each: at a unit boundary the rings refill at once, and those TMA
+// writes compete with the first MMAs of the next unit for shared memory; five
+// stages were measured 1-6 % slower.
+constexpr int kPKStages = 3, kPVStages = 3;
 
 struct PairLay {
   static constexpr uint32_t kQBox = kBM * 128;          // 128 rows x 64 bf16
@@ -854,12 +857,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   auto leader_bar = [&](int i) { return mapa_shared(bar(i), 0); };
-  auto peer_bar = [&](int i) { return mapa_shared(bar(i), 1); };
   // commit to the same barrier in both CTAs
-  auto commit_both = [&](int i) {
-    umma_commit_pair(leader_bar(i));
-    umma_commit_pair(peer_bar(i));
-  };
+  auto commit_both = [&](int i) { umma_commit_pair_both(bar(i)); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 

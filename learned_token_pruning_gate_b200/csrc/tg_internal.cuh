@@ -509,6 +509,16 @@ __device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// One commit that arrives on the barrier at this shared-memory offset in both
+// CTAs of the pair (CTA mask 0b11) once the pair's prior tcgen05 ops complete:
+// half the commits of one per CTA, each of which costs the tensor pipe ~64 cycles.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar_local) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar_local),
+      "h"(static_cast<uint16_t>(0x3))
+      : "memory");
+}
 // Arrive on a (possibly peer) barrier once the pair's prior tcgen05 ops complete.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
   asm volatile(
