@@ -39,9 +39,10 @@ constexpr int kPrepThreads = 256;
 constexpr int kScanRows = 16;      // state rows per scan CTA
 constexpr int kScanThreads = 256;
 
-// One workspace record per (chunk, head): W_k, Q_e and K~ as [kC][DH] fp32
-// (contiguous: the scan loads them with one bulk copy), U_v and O_v as
-// [DH / kScanRows][kC][kScanRows] (each scan block's columns contiguous), g_C.
+// One workspace record per (chunk, head), fp32: W_k and Q_e transposed, [DH][kC]
+// (the scan reads 4 consecutive chunk rows of one column at once), K~ as
+// [kC][DH], U_v and O_v as [DH / kScanRows][kC][kScanRows] (each scan block's
+// columns contiguous), g_C.
 template <int DH>
 struct ChunkRec {
   static constexpr int kMat = kC * DH;
@@ -78,12 +79,6 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return
 
 __device__ __forceinline__ void store_out(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store_out(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
-
-// a . b added to a pair of partial sums (packed fp32x2 FMAs: half the instructions)
-__device__ __forceinline__ float2 dot4x2(float4 a, float4 b, float2 acc) {
-  acc = __ffma2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y), acc);
-  return __ffma2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w), acc);
-}
 
 template <int DH>
 struct PrepLay {
@@ -322,10 +317,16 @@ __global__ void __launch_bounds__(kPrepThreads, 2) delta_chunk_prep_kernel(
       for (int s = t & ~3; s < t; ++s) a0 = fmaf(-arow[s], x[s], a0);
       x[t] = (a0 + a1) + (a2 + a3);
     }
+    if (wk) {  // W_k^T: this column's chunk rows are contiguous
+#pragma unroll
+      for (int t = 0; t < kC; t += 4)
+        *reinterpret_cast<float4*>(rec + R::kWk + c * kC + t) =
+            make_float4(x[t], x[t + 1], x[t + 2], x[t + 3]);
+    }
+    float qe4[4];
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
-      if (wk) rec[R::kWk + t * DH + c] = x[t];
-      else rec[R::kUv + R::blocked(t, c)] = x[t];
+      if (!wk) rec[R::kUv + R::blocked(t, c)] = x[t];
       const float* mrow = sM + t * LC;
       float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
@@ -339,162 +340,287 @@ __global__ void __launch_bounds__(kPrepThreads, 2) delta_chunk_prep_kernel(
 #pragma unroll
       for (int s = (t + 1) & ~3; s <= t; ++s) a0 = fmaf(mrow[s], x[s], a0);
       const float acc = (a0 + a1) + (a2 + a3);
-      if (wk) rec[R::kQe + t * DH + c] = fmaf(sGam[t], sQ[t * LD + c], -acc);
-      else rec[R::kOv + R::blocked(t, c)] = acc;
+      if (wk) {  // Q_e^T, four chunk rows per store
+        qe4[t & 3] = fmaf(sGam[t], sQ[t * LD + c], -acc);
+        if ((t & 3) == 3)
+          *reinterpret_cast<float4*>(rec + R::kQe + c * kC + t - 3) =
+              make_float4(qe4[0], qe4[1], qe4[2], qe4[3]);
+      } else {
+        rec[R::kOv + R::blocked(t, c)] = acc;
+      }
     }
   }
   if (tid == 0) rec[R::kG] = n > 0 ? sGam[n - 1] : 1.0f;
 }
 
+// Scan CTA (prompt, head, block of kScanRows state rows), per chunk:
+//   1. X = W_k S^T and Y = Q_e S^T for the block's rows: a thread owns 4 chunk
+//      rows x 4 state rows of both over a quarter of d (W_k^T, Q_e^T and the
+//      transposed state give it a float4 of each per d), then the quarters are
+//      summed; D = U_v - X goes to shared memory, O_v + Y to the output.
+//   2. S <- g_C S + D^T K~: a thread owns 4 state rows x 4 columns over a share
+//      of the chunk rows, the shares are summed by the threads that keep S in
+//      registers across chunks, which also write S^T for the next chunk.
+// W_k^T and Q_e^T of the next chunk load (one bulk copy) while this chunk's
+// update runs; K~ and the U_v / O_v columns are double-buffered.
 template <int DH>
 struct ScanLay {
-  static constexpr int LS = DH + 4;               // state rows (padded: 16 rows read at once)
-  static constexpr int kMat = kC * DH;            // W_k, Q_e, K~ unpadded
-  static constexpr int kStage = 3 * kMat + 2 * kC * kScanRows;  // + U_v, O_v columns
-  static constexpr int kS = 2 * kStage;
-  static constexpr int kD = kS + kScanRows * LS;  // [kC][kScanRows + 1]
-  static constexpr int kFloats = kD + kC * (kScanRows + 1);
+  static constexpr int R = kScanRows;
+  static constexpr int kWQ = 0;                       // W_k^T, Q_e^T: [2][DH][kC]
+  static constexpr int kK = kWQ + 2 * DH * kC;        // K~: [2 buffers][kC][DH]
+  static constexpr int kUO = kK + 2 * kC * DH;        // U_v, O_v columns: [2 buffers][2][kC][R]
+  static constexpr int kSt = kUO + 2 * 2 * kC * R;    // S^T of the block: [DH][R]
+  static constexpr int LDD = R + 4;                   // D pitch (float4 rows)
+  static constexpr int kD = kSt + DH * R;             // D = U_v - X: [kC][LDD]
+  static constexpr int kUpd = 4 * (DH / 4);           // update threads per chunk-row share
+  static constexpr int kTs = kScanThreads / kUpd;     // shares (2 at d = 128, 4 at d = 64)
+  static constexpr int kRedXY = 3 * 64 * 32;          // partial X, Y of quarters 1..3
+  static constexpr int kRedS = (kTs - 1) * kUpd * 16; // partial updates of shares 1..
+  static constexpr int kRed = kD + kC * LDD;
+  static constexpr int kFloats = kRed + (kRedXY > kRedS ? kRedXY : kRedS);
   static constexpr size_t kBytes = static_cast<size_t>(kFloats) * 4;
+  static_assert(kScanThreads == 256 && kC == 64 && R == 16, "thread mapping");
+  static_assert(kBytes <= 227 * 1024, "shared memory");
 };
 
 template <typename T, int DH>
-__global__ void __launch_bounds__(kScanThreads) delta_chunk_scan_kernel(
+__global__ void __launch_bounds__(kScanThreads, 1) delta_chunk_scan_kernel(
     T* __restrict__ out, const __grid_constant__ ChunkParams p) {
   using L = ScanLay<DH>;
   using R = ChunkRec<DH>;
-  constexpr int LS = L::LS;
-  constexpr int NC = DH / 16;  // state columns per thread in the update (4 or 8)
+  constexpr int RS = kScanRows;
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
-  float* sS = sm + L::kS;
+  float* sWT = sm + L::kWQ;
+  float* sQT = sWT + DH * kC;
+  float* sSt = sm + L::kSt;
   float* sD = sm + L::kD;
+  float* sRed = sm + L::kRed;
   const int tid = threadIdx.x;
-  const int i0 = blockIdx.x * kScanRows, h = blockIdx.y, b = blockIdx.z, H = p.heads;
+  const int i0 = blockIdx.x * RS, h = blockIdx.y, b = blockIdx.z, H = p.heads;
   const int c_first = p.chunk_start[b], n_chunks = p.chunk_start[b + 1] - c_first;
   const int row0 = p.kept_start[b], len = p.kept_start[b + 1] - row0;
-  __shared__ uint64_t s_full[2];  // stage s holds chunks s, s + 2, ...
+  __shared__ uint64_t s_wq, s_k[2];  // W_k^T, Q_e^T and the U_v / O_v columns; K~ per buffer
   __shared__ int s_abort;
   if (tid == 0) {
-    mbar_init(smem_u32(&s_full[0]), 1);
-    mbar_init(smem_u32(&s_full[1]), 1);
+    mbar_init(smem_u32(&s_wq), 1);
+    mbar_init(smem_u32(&s_k[0]), 1);
+    mbar_init(smem_u32(&s_k[1]), 1);
     s_abort = 0;
     mbar_fence_init();
   }
-  __syncthreads();
-
-  // Thread 0: chunk c's W_k, Q_e and K~ (one bulk copy) and this block's U_v and
-  // O_v columns (one each) into stage c & 1.  Every thread has finished reading
-  // that stage (the barrier at the end of the previous chunk).
-  constexpr uint32_t kMatsBytes = 3 * R::kMat * 4, kSliceBytes = R::kSlice * 4;
-  auto load_chunk = [&](int c) {
-    const float* rec = p.ws + (static_cast<size_t>(c_first + c) * H + h) * R::kFloats;
-    const uint32_t sb = smem_u32(sm + (c & 1) * L::kStage), bar = smem_u32(&s_full[c & 1]);
+  auto rec_of = [&](int c) { return p.ws + (static_cast<size_t>(c_first + c) * H + h) * R::kFloats; };
+  // Thread 0 issues the loads; every thread has finished reading the target
+  // buffer (a barrier precedes each call).
+  int wq_loads = 0, k_loads[2] = {0, 0};  // thread 0: for the drain after an abort
+  constexpr uint32_t kWQBytes = 2 * DH * kC * 4, kKBytes = kC * DH * 4, kSliceBytes = R::kSlice * 4;
+  auto load_wq = [&](int c) {
+    const float* rec = rec_of(c);
+    const uint32_t bar = smem_u32(&s_wq);
+    float* uo = sm + L::kUO + (c & 1) * 2 * kC * RS;
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar, kMatsBytes + 2 * kSliceBytes);
-    bulk_g2s(sb, rec, kMatsBytes, bar);
-    bulk_g2s(sb + kMatsBytes, rec + R::kUv + blockIdx.x * R::kSlice, kSliceBytes, bar);
-    bulk_g2s(sb + kMatsBytes + kSliceBytes, rec + R::kOv + blockIdx.x * R::kSlice, kSliceBytes, bar);
+    mbar_arrive_expect_tx(bar, kWQBytes + 2 * kSliceBytes);
+    bulk_g2s(smem_u32(sWT), rec + R::kWk, kWQBytes, bar);  // W_k^T and Q_e^T are adjacent
+    bulk_g2s(smem_u32(uo), rec + R::kUv + blockIdx.x * R::kSlice, kSliceBytes, bar);
+    bulk_g2s(smem_u32(uo + kC * RS), rec + R::kOv + blockIdx.x * R::kSlice, kSliceBytes, bar);
+    ++wq_loads;
+  };
+  auto load_k = [&](int c) {
+    const uint32_t bar = smem_u32(&s_k[c & 1]);
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, kKBytes);
+    bulk_g2s(smem_u32(sm + L::kK + (c & 1) * kC * DH), rec_of(c) + R::kKt, kKBytes, bar);
+    ++k_loads[c & 1];
   };
 
-  // update mapping: thread owns state row ru and the float4 column groups
-  // cu + 64 m (m < NC / 4): the 16 threads of a row read 16 consecutive float4
-  // of a K~ row (two bank-conflict-free wavefronts per load)
-  const int ru = tid >> 4, cu = (tid & 15) * 4;
-  // product mapping: thread owns chunk rows tg + 16 i (i < 4) of state row rp: a
-  // warp reads two consecutive rows of W_k / Q_e at once (a broadcast)
-  const int tg = tid >> 4, rp = tid & 15;
-  float sreg[NC];
+  // product mapping: quarter dq of d; within it, a warp covers 8 chunk-row groups
+  // (4 rows each, consecutive) x 4 state-row groups (4 rows each)
+  const int dq = tid >> 6, w64 = tid & 63;
+  const int tq = ((w64 >> 5) << 3) | (w64 & 7), rq = (w64 >> 3) & 3;
+  // update mapping: share ts of the chunk rows; a warp covers consecutive
+  // column groups of one (d = 128) or two (d = 64) state-row groups
+  constexpr int kCq = DH / 4;
+  const int ts = tid / L::kUpd, u = tid % L::kUpd;
+  const int cq = u % kCq, ru = u / kCq;
+  float sreg[16];  // S rows 4 ru + i, columns 4 cq + j (threads of share 0)
 #pragma unroll
-  for (int j = 0; j < NC; ++j) sreg[j] = 0.0f;
-#pragma unroll
-  for (int m = 0; m < NC / 4; ++m)
-    *reinterpret_cast<float4*>(sS + ru * LS + cu + 64 * m) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  if (tid == 0 && n_chunks > 0) load_chunk(0);
-  int loaded = n_chunks > 0 ? 1 : 0;  // chunks whose load was issued
+  for (int e = 0; e < 16; ++e) sreg[e] = 0.0f;
+  for (int e = tid; e < DH * RS; e += kScanThreads) sSt[e] = 0.0f;
+  __syncthreads();
+  if (tid == 0 && n_chunks > 0) {
+    load_wq(0);
+    load_k(0);
+    if (n_chunks > 1) load_k(1);
+  }
   bool ok = true;
   for (int c = 0; c < n_chunks; ++c) {
-    if (tid == 0 && c + 1 < n_chunks) load_chunk(c + 1);
-    loaded = min(c + 2, n_chunks);
-    const bool landed =
-        mbar_wait(smem_u32(&s_full[c & 1]), (c >> 1) & 1, &s_abort, p.status, kDevTimeoutDelta);
-    if (__syncthreads_or(!landed)) {  // one way out for the whole CTA
+    const float* uo = sm + L::kUO + (c & 1) * 2 * kC * RS;
+    const float* sUv = uo;
+    const float* sOv = uo + kC * RS;
+    const float* sKt = sm + L::kK + (c & 1) * kC * DH;
+    const float gC = __ldg(rec_of(c) + R::kG);
+    // ---- X and Y ------------------------------------------------------------
+    bool landed = mbar_wait(smem_u32(&s_wq), c & 1, &s_abort, p.status, kDevTimeoutDelta);
+    if (__syncthreads_or(!landed)) {
       ok = false;
       break;
     }
-    const float* st = sm + (c & 1) * L::kStage;
-    const float* sW = st;
-    const float* sQe = st + R::kMat;
-    const float* sKt = st + 2 * R::kMat;
-    const float* sUv = st + 3 * R::kMat;
-    const float* sOv = sUv + kC * kScanRows;
-    const float gC = __ldg(p.ws + (static_cast<size_t>(c_first + c) * H + h) * R::kFloats + R::kG);
-    // X = W_k S^T and Y = Q_e S^T for this thread's 4 chunk rows and state row rp
-    float2 ax2[4], ay2[4];
+    float2 ax[4][2], ay[4][2];  // [chunk row i][state rows (2 jp, 2 jp + 1)]
 #pragma unroll
-    for (int i = 0; i < 4; ++i) ax2[i] = ay2[i] = make_float2(0.0f, 0.0f);
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int jp = 0; jp < 2; ++jp) ax[i][jp] = ay[i][jp] = make_float2(0.0f, 0.0f);
+    {
+      constexpr int kDq = DH / 4;
+      const float* wt = sWT + (dq * kDq) * kC + 4 * tq;
+      const float* qt = sQT + (dq * kDq) * kC + 4 * tq;
+      const float* st = sSt + (dq * kDq) * RS + 4 * rq;
 #pragma unroll 4
-    for (int d = 0; d < DH; d += 4) {
-      const float4 s4 = *reinterpret_cast<const float4*>(sS + rp * LS + d);
+      for (int d = 0; d < kDq; ++d) {
+        const float4 w4 = *reinterpret_cast<const float4*>(wt + d * kC);
+        const float4 q4 = *reinterpret_cast<const float4*>(qt + d * kC);
+        const float4 s4 = *reinterpret_cast<const float4*>(st + d * RS);
+        const float2 s01 = make_float2(s4.x, s4.y), s23 = make_float2(s4.z, s4.w);
+        const float wv[4] = {w4.x, w4.y, w4.z, w4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ax[i][0] = __ffma2_rn(make_float2(wv[i], wv[i]), s01, ax[i][0]);
+          ax[i][1] = __ffma2_rn(make_float2(wv[i], wv[i]), s23, ax[i][1]);
+          ay[i][0] = __ffma2_rn(make_float2(qv[i], qv[i]), s01, ay[i][0]);
+          ay[i][1] = __ffma2_rn(make_float2(qv[i], qv[i]), s23, ay[i][1]);
+        }
+      }
+    }
+    // quarters 1..3 hand their partial sums to quarter 0 (one column per value:
+    // consecutive threads, consecutive words)
+    if (dq > 0) {
+      float* red = sRed + (dq - 1) * 32 * 64 + w64;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jp = 0; jp < 2; ++jp) {
+          red[((i * 2 + jp) * 2 + 0) * 64] = ax[i][jp].x;
+          red[((i * 2 + jp) * 2 + 1) * 64] = ax[i][jp].y;
+          red[(16 + (i * 2 + jp) * 2 + 0) * 64] = ay[i][jp].x;
+          red[(16 + (i * 2 + jp) * 2 + 1) * 64] = ay[i][jp].y;
+        }
+    }
+    __syncthreads();  // W_k^T and Q_e^T are read: the next chunk's may load
+    if (tid == 0 && c + 1 < n_chunks) load_wq(c + 1);
+    if (dq == 0) {
+#pragma unroll
+      for (int q3 = 0; q3 < 3; ++q3) {
+        const float* red = sRed + q3 * 32 * 64 + w64;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int jp = 0; jp < 2; ++jp) {
+            ax[i][jp].x += red[((i * 2 + jp) * 2 + 0) * 64];
+            ax[i][jp].y += red[((i * 2 + jp) * 2 + 1) * 64];
+            ay[i][jp].x += red[(16 + (i * 2 + jp) * 2 + 0) * 64];
+            ay[i][jp].y += red[(16 + (i * 2 + jp) * 2 + 1) * 64];
+          }
+      }
+      const int t0 = c * kC;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        ax2[i] = dot4x2(*reinterpret_cast<const float4*>(sW + (tg + 16 * i) * DH + d), s4, ax2[i]);
-        ay2[i] = dot4x2(*reinterpret_cast<const float4*>(sQe + (tg + 16 * i) * DH + d), s4, ay2[i]);
+        const int t = 4 * tq + i;
+        const float4 uv = *reinterpret_cast<const float4*>(sUv + t * RS + 4 * rq);
+        const float4 ov = *reinterpret_cast<const float4*>(sOv + t * RS + 4 * rq);
+        *reinterpret_cast<float4*>(sD + t * L::LDD + 4 * rq) =
+            make_float4(uv.x - ax[i][0].x, uv.y - ax[i][0].y, uv.z - ax[i][1].x, uv.w - ax[i][1].y);
+        if (t0 + t < len) {
+          T* o = out + (static_cast<size_t>(row0 + t0 + t) * H + h) * DH + i0 + 4 * rq;
+          store_out(o + 0, ov.x + ay[i][0].x);
+          store_out(o + 1, ov.y + ay[i][0].y);
+          store_out(o + 2, ov.z + ay[i][1].x);
+          store_out(o + 3, ov.w + ay[i][1].y);
+        }
       }
     }
-    float ax[4], ay[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ax[i] = ax2[i].x + ax2[i].y;
-      ay[i] = ay2[i].x + ay2[i].y;
+    // ---- S <- g_C S + D^T K~ ---------------------------------------------------
+    landed = mbar_wait(smem_u32(&s_k[c & 1]), (c >> 1) & 1, &s_abort, p.status, kDevTimeoutDelta);
+    if (__syncthreads_or(!landed)) {  // also: D is complete
+      ok = false;
+      break;
     }
-    const int t0 = c * kC;  // chunk rows within the prompt
+    float2 acc[4][2];  // [state row i][columns (2 jp, 2 jp + 1)]
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = tg + 16 * i;
-      sD[t * (kScanRows + 1) + rp] = sUv[t * kScanRows + rp] - ax[i];
-      if (t0 + t < len)
-        store_out(out + (static_cast<size_t>(row0 + t0 + t) * H + h) * DH + i0 + rp,
-                  sOv[t * kScanRows + rp] + ay[i]);
-    }
-    __syncthreads();
-    // S <- g_C S + (U_v - X)^T K~ for this thread's row and columns
-#pragma unroll
-    for (int j = 0; j < NC; ++j) sreg[j] *= gC;
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = make_float2(0.0f, 0.0f);
+    {
+      constexpr int kTper = kC / L::kTs;
+      const float* dr = sD + (ts * kTper) * L::LDD + 4 * ru;
+      const float* kr = sKt + (ts * kTper) * DH + 4 * cq;
 #pragma unroll 4
-    for (int t = 0; t < kC; ++t) {
-      const float dd = sD[t * (kScanRows + 1) + ru];
-      const float2 d2 = make_float2(dd, dd);
+      for (int t = 0; t < kTper; ++t) {
+        const float4 d4 = *reinterpret_cast<const float4*>(dr + t * L::LDD);
+        const float4 k4 = *reinterpret_cast<const float4*>(kr + t * DH);
+        const float2 k01 = make_float2(k4.x, k4.y), k23 = make_float2(k4.z, k4.w);
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-      for (int m = 0; m < NC / 4; ++m) {
-        const float4 kt = *reinterpret_cast<const float4*>(sKt + t * DH + cu + 64 * m);
-        const float2 lo = __ffma2_rn(d2, make_float2(kt.x, kt.y), make_float2(sreg[4 * m], sreg[4 * m + 1]));
-        const float2 hi = __ffma2_rn(d2, make_float2(kt.z, kt.w), make_float2(sreg[4 * m + 2], sreg[4 * m + 3]));
-        sreg[4 * m] = lo.x;
-        sreg[4 * m + 1] = lo.y;
-        sreg[4 * m + 2] = hi.x;
-        sreg[4 * m + 3] = hi.y;
+        for (int i = 0; i < 4; ++i) {
+          acc[i][0] = __ffma2_rn(make_float2(dv[i], dv[i]), k01, acc[i][0]);
+          acc[i][1] = __ffma2_rn(make_float2(dv[i], dv[i]), k23, acc[i][1]);
+        }
       }
     }
+    if (ts > 0) {
+      float* red = sRed + (ts - 1) * 16 * L::kUpd + u;
 #pragma unroll
-    for (int m = 0; m < NC / 4; ++m)
-      *reinterpret_cast<float4*>(sS + ru * LS + cu + 64 * m) =
-          make_float4(sreg[4 * m], sreg[4 * m + 1], sreg[4 * m + 2], sreg[4 * m + 3]);
-    __syncthreads();  // state and stage free for the next chunk
+      for (int i = 0; i < 4; ++i) {
+        red[(i * 4 + 0) * L::kUpd] = acc[i][0].x;
+        red[(i * 4 + 1) * L::kUpd] = acc[i][0].y;
+        red[(i * 4 + 2) * L::kUpd] = acc[i][1].x;
+        red[(i * 4 + 3) * L::kUpd] = acc[i][1].y;
+      }
+    }
+    __syncthreads();  // K~ of this buffer is read: the chunk after next may load
+    if (tid == 0 && c + 2 < n_chunks) load_k(c + 2);
+    if (ts == 0) {
+#pragma unroll
+      for (int s2 = 1; s2 < L::kTs; ++s2) {
+        const float* red = sRed + (s2 - 1) * 16 * L::kUpd + u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i][0].x += red[(i * 4 + 0) * L::kUpd];
+          acc[i][0].y += red[(i * 4 + 1) * L::kUpd];
+          acc[i][1].x += red[(i * 4 + 2) * L::kUpd];
+          acc[i][1].y += red[(i * 4 + 3) * L::kUpd];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sreg[i * 4 + 0] = fmaf(gC, sreg[i * 4 + 0], acc[i][0].x);
+        sreg[i * 4 + 1] = fmaf(gC, sreg[i * 4 + 1], acc[i][0].y);
+        sreg[i * 4 + 2] = fmaf(gC, sreg[i * 4 + 2], acc[i][1].x);
+        sreg[i * 4 + 3] = fmaf(gC, sreg[i * 4 + 3], acc[i][1].y);
+      }
+      // S^T for the next chunk's products: column 4 cq + j, rows 4 ru .. 4 ru + 3
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4*>(sSt + (4 * cq + j) * RS + 4 * ru) =
+            make_float4(sreg[j], sreg[4 + j], sreg[8 + j], sreg[12 + j]);
+    }
+    __syncthreads();  // S^T complete; the reduction buffer is free
   }
   if (!ok) {
     // a load did not land in time: wait (bounded) for every load in flight before
     // the shared memory is released; the outputs are undefined
-    if (tid == 0)
-      for (int c = 0; c < loaded; ++c) mbar_drain(smem_u32(&s_full[c & 1]), (c >> 1) & 1);
+    if (tid == 0) {
+      if (wq_loads > 0) mbar_drain(smem_u32(&s_wq), (wq_loads - 1) & 1);
+      for (int kb = 0; kb < 2; ++kb)
+        if (k_loads[kb] > 0) mbar_drain(smem_u32(&s_k[kb]), (k_loads[kb] - 1) & 1);
+    }
     __syncthreads();
     return;
   }
-  if (p.state) {
-    float* dst = p.state + ((static_cast<size_t>(b) * H + h) * DH + i0 + ru) * DH + cu;
+  if (p.state && ts == 0) {
 #pragma unroll
-    for (int m = 0; m < NC / 4; ++m)
-      *reinterpret_cast<float4*>(dst + 64 * m) =
-          make_float4(sreg[4 * m], sreg[4 * m + 1], sreg[4 * m + 2], sreg[4 * m + 3]);
+    for (int i = 0; i < 4; ++i) {
+      float* dst = p.state + ((static_cast<size_t>(b) * H + h) * DH + i0 + 4 * ru + i) * DH + 4 * cq;
+      *reinterpret_cast<float4*>(dst) =
+          make_float4(sreg[i * 4 + 0], sreg[i * 4 + 1], sreg[i * 4 + 2], sreg[i * 4 + 3]);
+    }
   }
 }
 
