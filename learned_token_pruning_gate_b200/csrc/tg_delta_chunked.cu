@@ -164,23 +164,23 @@ __global__ void __launch_bounds__(kPrepThreads, 2) delta_chunk_prep_kernel(
   const int n = min(kC, p.kept_start[b + 1] - r0);
   float* rec = p.ws + (static_cast<size_t>(g) * H + h) * R::kFloats;
 
-  // rows of q and k as fp32 (16-byte loads), zero past the chunk's end
+  // rows of q and k (16-byte loads, all in flight at once), normalised on the
+  // way into shared memory: k^ = k / sqrt(|k|^2 + eps), q^ = q / sqrt(|q|^2 + eps)
+  // / sqrt(d).  A row's vectors sit in kVecRow consecutive lanes, so its squared
+  // norm is a shuffle reduction.  Rows past the chunk's end are zero.
   constexpr int kVecRow = DH / V::kN;
-  for (int idx = tid; idx < kC * kVecRow; idx += kPrepThreads) {
+  constexpr int kIters = kC * kVecRow / kPrepThreads;
+  static_assert(kC * kVecRow % kPrepThreads == 0 && 32 % kVecRow == 0, "row vectors per warp");
+  uint4 ku[kIters], qu[kIters];
+#pragma unroll
+  for (int u = 0; u < kIters; ++u) {
+    const int idx = tid + u * kPrepThreads;
     const int t = idx / kVecRow, c = (idx - t * kVecRow) * V::kN;
-    float fk[V::kN], fq[V::kN];
+    ku[u] = qu[u] = make_uint4(0u, 0u, 0u, 0u);
     if (t < n) {
       const size_t off = (static_cast<size_t>(r0 + t) * H + h) * DH + c;
-      V::to_f32(__ldg(reinterpret_cast<const uint4*>(k + off)), fk);
-      V::to_f32(__ldg(reinterpret_cast<const uint4*>(q + off)), fq);
-    } else {
-#pragma unroll
-      for (int e = 0; e < V::kN; ++e) fk[e] = fq[e] = 0.0f;
-    }
-#pragma unroll
-    for (int e = 0; e < V::kN; e += 4) {
-      *reinterpret_cast<float4*>(sK + t * LD + c + e) = make_float4(fk[e], fk[e + 1], fk[e + 2], fk[e + 3]);
-      *reinterpret_cast<float4*>(sQ + t * LD + c + e) = make_float4(fq[e], fq[e + 1], fq[e + 2], fq[e + 3]);
+      ku[u] = __ldg(reinterpret_cast<const uint4*>(k + off));
+      qu[u] = __ldg(reinterpret_cast<const uint4*>(q + off));
     }
   }
   if (tid < kC) {
@@ -188,38 +188,61 @@ __global__ void __launch_bounds__(kPrepThreads, 2) delta_chunk_prep_kernel(
     sBeta[t] = t < n ? p.beta[static_cast<size_t>(r0 + t) * H + h] : 0.0f;
     sRho[t] = t < n ? p.log_alpha[static_cast<size_t>(r0 + t) * H + h] : 0.0f;  // log alpha, for now
   }
-  __syncthreads();
-  if (tid == 0) {
-    // prefix sums of the finite log alphas (fp64) and counts of alpha = 0 rows
-    double P = 0.0;
-    int ninf = 0;
-    for (int t = 0; t < kC; ++t) {
-      const float la = sRho[t];
-      if (la == -INFINITY) ++ninf;
-      else P += static_cast<double>(la);
-      sP[t] = P;
-      sNinf[t] = ninf;
-    }
-  }
-  __syncthreads();
-  // row norms: k^ = k / sqrt(|k|^2 + eps), q^ = q / sqrt(|q|^2 + eps) / sqrt(d)
-  for (int t = warp; t < n; t += kPrepThreads / 32) {
+#pragma unroll
+  for (int u = 0; u < kIters; ++u) {
+    const int idx = tid + u * kPrepThreads;
+    const int t = idx / kVecRow, c = (idx - t * kVecRow) * V::kN;
+    float fk[V::kN], fq[V::kN];
+    V::to_f32(ku[u], fk);
+    V::to_f32(qu[u], fq);
     float ssk = 0.0f, ssq = 0.0f;
-    for (int c = lane; c < DH; c += 32) {
-      ssk = fmaf(sK[t * LD + c], sK[t * LD + c], ssk);
-      ssq = fmaf(sQ[t * LD + c], sQ[t * LD + c], ssq);
+#pragma unroll
+    for (int e = 0; e < V::kN; ++e) {
+      ssk = fmaf(fk[e], fk[e], ssk);
+      ssq = fmaf(fq[e], fq[e], ssq);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int o = kVecRow / 2; o > 0; o >>= 1) {
       ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
       ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
     }
-    const float ik = rsqrtf(ssk + p.eps), iq = rsqrtf(ssq + p.eps) * p.q_scale;
-    for (int c = lane; c < DH; c += 32) {
-      sK[t * LD + c] *= ik;
-      sQ[t * LD + c] *= iq;
+    // rows past the chunk's end stay zero (with eps = 0 their scale would be inf)
+    const float ik = t < n ? rsqrtf(ssk + p.eps) : 0.0f;
+    const float iq = t < n ? rsqrtf(ssq + p.eps) * p.q_scale : 0.0f;
+#pragma unroll
+    for (int e = 0; e < V::kN; e += 4) {
+      *reinterpret_cast<float4*>(sK + t * LD + c + e) =
+          make_float4(fk[e] * ik, fk[e + 1] * ik, fk[e + 2] * ik, fk[e + 3] * ik);
+      *reinterpret_cast<float4*>(sQ + t * LD + c + e) =
+          make_float4(fq[e] * iq, fq[e + 1] * iq, fq[e + 2] * iq, fq[e + 3] * iq);
     }
   }
+  __syncthreads();
+  if (warp == 0) {
+    // prefix sums of the finite log alphas (fp64) and counts of alpha = 0 rows:
+    // two rows per lane, then a scan over the warp
+    static_assert(kC == 64, "two chunk rows per lane");
+    const float l0 = sRho[2 * lane], l1 = sRho[2 * lane + 1];
+    const double d0 = l0 == -INFINITY ? 0.0 : static_cast<double>(l0);
+    const double d1 = l1 == -INFINITY ? 0.0 : static_cast<double>(l1);
+    const int i0 = l0 == -INFINITY ? 1 : 0, i1 = l1 == -INFINITY ? 1 : 0;
+    double P = d0 + d1;
+    int ni = i0 + i1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double yP = __shfl_up_sync(0xffffffffu, P, o);
+      const int yn = __shfl_up_sync(0xffffffffu, ni, o);
+      if (lane >= o) {
+        P += yP;
+        ni += yn;
+      }
+    }
+    sP[2 * lane] = P - d1;
+    sP[2 * lane + 1] = P;
+    sNinf[2 * lane] = ni - i1;
+    sNinf[2 * lane + 1] = ni;
+  }
+  __syncthreads();
   // g_t (decay from the chunk's start through t) and g_{n-1} / g_t
   if (tid < kC) {
     const int t = tid;
