@@ -397,7 +397,7 @@ struct ScanLay {
   static constexpr int kD = kSt + DH * R;             // D = U_v - X: [kC][LDD]
   static constexpr int kUpd = 4 * (DH / 4);           // update threads per chunk-row share
   static constexpr int kTs = kScanThreads / kUpd;     // shares (2 at d = 128, 4 at d = 64)
-  static constexpr int kRedXY = 3 * 64 * 32;          // partial X, Y of quarters 1..3
+  static constexpr int kRedXY = 4 * 64 * 32;          // partial X, Y of the four quarters
   static constexpr int kRedS = (kTs - 1) * kUpd * 16; // partial updates of shares 1..
   static constexpr int kRed = kD + kC * LDD;
   static constexpr int kFloats = kRed + (kRedXY > kRedS ? kRedXY : kRedS);
@@ -514,10 +514,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) delta_chunk_scan_kernel(
         }
       }
     }
-    // quarters 1..3 hand their partial sums to quarter 0 (one column per value:
-    // consecutive threads, consecutive words)
-    if (dq > 0) {
-      float* red = sRed + (dq - 1) * 32 * 64 + w64;
+    // every quarter hands its partial sums over (one column per value:
+    // consecutive threads, consecutive words); quarter dq then finishes chunk
+    // row 4 tq + dq of the block, summing the four quarters' partials
+    {
+      float* red = sRed + dq * 32 * 64 + w64;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -530,35 +531,28 @@ __global__ void __launch_bounds__(kScanThreads, 1) delta_chunk_scan_kernel(
     }
     __syncthreads();  // W_k^T and Q_e^T are read: the next chunk's may load
     if (tid == 0 && c + 1 < n_chunks) load_wq(c + 1);
-    if (dq == 0) {
+    {
+      float xs[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ys[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int q3 = 0; q3 < 3; ++q3) {
-        const float* red = sRed + q3 * 32 * 64 + w64;
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float* red = sRed + q4 * 32 * 64 + w64;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int jp = 0; jp < 2; ++jp) {
-            ax[i][jp].x += red[((i * 2 + jp) * 2 + 0) * 64];
-            ax[i][jp].y += red[((i * 2 + jp) * 2 + 1) * 64];
-            ay[i][jp].x += red[(16 + (i * 2 + jp) * 2 + 0) * 64];
-            ay[i][jp].y += red[(16 + (i * 2 + jp) * 2 + 1) * 64];
-          }
-      }
-      const int t0 = c * kC;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = 4 * tq + i;
-        const float4 uv = *reinterpret_cast<const float4*>(sUv + t * RS + 4 * rq);
-        const float4 ov = *reinterpret_cast<const float4*>(sOv + t * RS + 4 * rq);
-        *reinterpret_cast<float4*>(sD + t * L::LDD + 4 * rq) =
-            make_float4(uv.x - ax[i][0].x, uv.y - ax[i][0].y, uv.z - ax[i][1].x, uv.w - ax[i][1].y);
-        if (t0 + t < len) {
-          T* o = out + (static_cast<size_t>(row0 + t0 + t) * H + h) * DH + i0 + 4 * rq;
-          store_out(o + 0, ov.x + ay[i][0].x);
-          store_out(o + 1, ov.y + ay[i][0].y);
-          store_out(o + 2, ov.z + ay[i][1].x);
-          store_out(o + 3, ov.w + ay[i][1].y);
+        for (int e = 0; e < 4; ++e) {  // state row 4 rq + e: accumulator (dq * 2 + e / 2) * 2 + e % 2
+          xs[e] += red[(dq * 4 + e) * 64];
+          ys[e] += red[(16 + dq * 4 + e) * 64];
         }
+      }
+      const int t = 4 * tq + dq, t0 = c * kC;
+      const float4 uv = *reinterpret_cast<const float4*>(sUv + t * RS + 4 * rq);
+      const float4 ov = *reinterpret_cast<const float4*>(sOv + t * RS + 4 * rq);
+      *reinterpret_cast<float4*>(sD + t * L::LDD + 4 * rq) =
+          make_float4(uv.x - xs[0], uv.y - xs[1], uv.z - xs[2], uv.w - xs[3]);
+      if (t0 + t < len) {
+        T* o = out + (static_cast<size_t>(row0 + t0 + t) * H + h) * DH + i0 + 4 * rq;
+        store_out(o + 0, ov.x + ys[0]);
+        store_out(o + 1, ov.y + ys[1]);
+        store_out(o + 2, ov.z + ys[2]);
+        store_out(o + 3, ov.w + ys[3]);
       }
     }
     // ---- S <- g_C S + D^T K~ ---------------------------------------------------
