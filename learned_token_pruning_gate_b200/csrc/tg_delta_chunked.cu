@@ -70,13 +70,6 @@ struct ChunkParams {
   float q_scale;  // 1 / sqrt(d)
 };
 
-template <typename T>
-__device__ __forceinline__ float to_f32(T x);
-template <>
-__device__ __forceinline__ float to_f32<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
-
 __device__ __forceinline__ void store_out(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store_out(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
@@ -307,22 +300,50 @@ __global__ void __launch_bounds__(kPrepThreads, 2) delta_chunk_prep_kernel(
   // O_v = M U_v; threads [DH, 2 DH) solve (I + A) W_k = diag(beta g) K^ and form
   // Q_e = diag(g) Q^ - M W_k (they also write K~ = diag(ratio(C, s)) K^ from their
   // column first).  Forward substitution: x_t = r_t - sum_{s<t} A_ts x_s.
-  if (tid < 2 * DH) {
-    const bool wk = tid >= DH;
-    const int c = wk ? tid - DH : tid;
-    float x[kC];
-    if (wk) {
+  // V reaches shared memory (over K^, once read) with coalesced 16-byte loads;
+  // W_k (over V, once read) and Q_e (over Q^, element by element) leave it for
+  // the record transposed, with coalesced stores.
+  const bool col = tid < 2 * DH, wk = tid >= DH;
+  const int c = wk ? tid - DH : tid;
+  float x[kC];
+  if (col && wk) {
 #pragma unroll
-      for (int t = 0; t < kC; ++t) {
-        const float e = sK[t * LD + c];
-        x[t] = sBeta[t] * sGam[t] * e;
-        rec[R::kKt + t * DH + c] = sRho[t] * e;
-      }
-    } else {
-#pragma unroll
-      for (int t = 0; t < kC; ++t)
-        x[t] = t < n ? sBeta[t] * to_f32(v[(static_cast<size_t>(r0 + t) * H + h) * DH + c]) : 0.0f;
+    for (int t = 0; t < kC; ++t) {
+      const float e = sK[t * LD + c];
+      x[t] = sBeta[t] * sGam[t] * e;
+      rec[R::kKt + t * DH + c] = sRho[t] * e;
     }
+  }
+  __syncthreads();  // K^ is read: its rows take V
+  float* sV = sK;
+  {
+    uint4 vu[kIters];
+#pragma unroll
+    for (int u = 0; u < kIters; ++u) {
+      const int idx = tid + u * kPrepThreads;
+      const int t = idx / kVecRow, cc = (idx - t * kVecRow) * V::kN;
+      vu[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (t < n)
+        vu[u] = __ldg(reinterpret_cast<const uint4*>(v + (static_cast<size_t>(r0 + t) * H + h) * DH + cc));
+    }
+#pragma unroll
+    for (int u = 0; u < kIters; ++u) {
+      const int idx = tid + u * kPrepThreads;
+      const int t = idx / kVecRow, cc = (idx - t * kVecRow) * V::kN;
+      float fv[V::kN];
+      V::to_f32(vu[u], fv);
+#pragma unroll
+      for (int e = 0; e < V::kN; e += 4)
+        *reinterpret_cast<float4*>(sV + t * LD + cc + e) = make_float4(fv[e], fv[e + 1], fv[e + 2], fv[e + 3]);
+    }
+  }
+  __syncthreads();
+  if (col && !wk) {
+#pragma unroll
+    for (int t = 0; t < kC; ++t) x[t] = sBeta[t] * sV[t * LD + c];  // zero past the chunk's end
+  }
+  __syncthreads();  // V is read: its rows take W_k
+  if (col) {
     // rows of A and M are the same for every thread: float4 broadcast reads
 #pragma unroll
     for (int t = 1; t < kC; ++t) {
@@ -340,13 +361,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2) delta_chunk_prep_kernel(
       for (int s = t & ~3; s < t; ++s) a0 = fmaf(-arow[s], x[s], a0);
       x[t] = (a0 + a1) + (a2 + a3);
     }
-    if (wk) {  // W_k^T: this column's chunk rows are contiguous
+    if (wk) {
 #pragma unroll
-      for (int t = 0; t < kC; t += 4)
-        *reinterpret_cast<float4*>(rec + R::kWk + c * kC + t) =
-            make_float4(x[t], x[t + 1], x[t + 2], x[t + 3]);
+      for (int t = 0; t < kC; ++t) sV[t * LD + c] = x[t];
     }
-    float qe4[4];
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
       if (!wk) rec[R::kUv + R::blocked(t, c)] = x[t];
@@ -363,15 +381,19 @@ __global__ void __launch_bounds__(kPrepThreads, 2) delta_chunk_prep_kernel(
 #pragma unroll
       for (int s = (t + 1) & ~3; s <= t; ++s) a0 = fmaf(mrow[s], x[s], a0);
       const float acc = (a0 + a1) + (a2 + a3);
-      if (wk) {  // Q_e^T, four chunk rows per store
-        qe4[t & 3] = fmaf(sGam[t], sQ[t * LD + c], -acc);
-        if ((t & 3) == 3)
-          *reinterpret_cast<float4*>(rec + R::kQe + c * kC + t - 3) =
-              make_float4(qe4[0], qe4[1], qe4[2], qe4[3]);
-      } else {
-        rec[R::kOv + R::blocked(t, c)] = acc;
-      }
+      if (wk) sQ[t * LD + c] = fmaf(sGam[t], sQ[t * LD + c], -acc);  // Q_e over Q^
+      else rec[R::kOv + R::blocked(t, c)] = acc;
     }
+  }
+  __syncthreads();
+  // W_k^T and Q_e^T: a thread takes four consecutive chunk rows of one column,
+  // so 16 consecutive threads write one 256-byte row of the transposed matrix
+  for (int i = tid; i < DH * (kC / 4); i += kPrepThreads) {
+    const int cc = i / (kC / 4), t4 = (i - cc * (kC / 4)) * 4;
+    *reinterpret_cast<float4*>(rec + R::kWk + cc * kC + t4) =
+        make_float4(sV[t4 * LD + cc], sV[(t4 + 1) * LD + cc], sV[(t4 + 2) * LD + cc], sV[(t4 + 3) * LD + cc]);
+    *reinterpret_cast<float4*>(rec + R::kQe + cc * kC + t4) =
+        make_float4(sQ[t4 * LD + cc], sQ[(t4 + 1) * LD + cc], sQ[(t4 + 2) * LD + cc], sQ[(t4 + 3) * LD + cc]);
   }
   if (tid == 0) rec[R::kG] = n > 0 ? sGam[n - 1] : 1.0f;
 }
