@@ -548,6 +548,66 @@ def run_ncu_case(args):
                       "M": layer.M}))
 
 
+def _library_baselines(layer, inp, w, res, timed):
+    """Library calls doing each stage's operation (or its main part) on the same
+    shapes and buffers, timed like the stages (L2 flushed, CUDA events): context
+    beside the stage times, never on the layer's path.  gate: the cuBLAS GEMM of
+    the residual with W1 alone (no GELU, w2 or bias); top-K: torch.topk over each
+    prompt's document span; gather: torch.index_select of the four tensors, and
+    one device copy of the same bytes; attention: PyTorch SDPA (cuDNN, flash)
+    causal over each prompt's kept rows, without the key bias.  The 1-element
+    add is the floor of this timing method."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+
+    h, q, k, v, W1 = res[0], res[1], res[2], res[3], res[4]
+    dev = h.device
+    out = {}
+    tiny = torch.zeros(1, device=dev)
+    out["floor_1_element_add_us"] = timed(lambda: tiny.add_(1), 20)
+    w1t = W1.t() if W1.shape[0] != h.shape[1] else W1
+    out["cublas_gemm_residual_w1_us"] = timed(lambda: torch.matmul(h, w1t), 20)
+    cu = np.asarray(inp.cu_seqlens)
+    spans = [(int(cu[b] + inp.doc_begin[b]), int(cu[b] + inp.doc_end[b]), int(kb))
+             for b, kb in enumerate(inp.budget)]
+    spans = [(a, e, min(kb, e - a)) for a, e, kb in spans if e > a and kb > 0]
+    z = layer.z
+    out["torch_topk_us"] = timed(lambda: [torch.topk(z[a:e], kb) for a, e, kb in spans], 20)
+    kept = layer.kept_idx.long()
+    M = int(kept.numel())
+    dst = [torch.empty((M,) + tuple(t.shape[1:]), dtype=t.dtype, device=dev) for t in (h, q, k, v)]
+    out["torch_index_select_x4_us"] = timed(
+        lambda: [torch.index_select(t, 0, kept, out=o) for t, o in zip((h, q, k, v), dst)], 20)
+    nb = sum(o.numel() * o.element_size() for o in dst)
+    c_src = torch.empty(nb, dtype=torch.uint8, device=dev)
+    c_dst = torch.empty_like(c_src)
+    out["torch_copy_same_bytes_us"] = timed(lambda: c_dst.copy_(c_src), 20)
+    del dst, c_src, c_dst
+    hq, hkv, dh = w.n_q_heads, w.n_kv_heads, w.head_dim
+    ck = np.asarray(layer.cu_kept_host)
+    per = []
+    for b in range(len(ck) - 1):
+        a, e = int(ck[b]), int(ck[b + 1])
+        if e <= a:
+            continue
+        heads = lambda t, n: t[a:e].reshape(e - a, n, dh).transpose(0, 1).unsqueeze(0)  # noqa: E731
+        per.append((heads(layer.q_c, hq).contiguous(),
+                    heads(layer.k_c, hkv).repeat_interleave(hq // hkv, dim=1).contiguous(),
+                    heads(layer.v_c, hkv).repeat_interleave(hq // hkv, dim=1).contiguous()))
+    for name, be in (("cudnn", SDPBackend.CUDNN_ATTENTION), ("flash", SDPBackend.FLASH_ATTENTION)):
+        key = f"sdpa_{name}_causal_no_bias_us"
+        try:
+            with sdpa_kernel([be]):
+                out[key] = timed(lambda: [F.scaled_dot_product_attention(a_, b_, c_, is_causal=True)
+                                          for a_, b_, c_ in per], 20)
+        except RuntimeError:
+            out[key] = None
+    del per
+    torch.cuda.synchronize()
+    return {key: (round(val, 2) if val is not None else None) for key, val in out.items()}
+
+
 def run_extras(args):
     """Supplementary layer-level figures for one workload (one JSON line; not the
     bench line): the bias overhead of the gated attention (logsig vs none), the
@@ -594,6 +654,7 @@ def run_extras(args):
     import ctypes
     st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     stage_us = {s: timed(lambda s=s: getattr(layer, s)(st), 20) for s in GatedLayer.STAGES}
+    library = _library_baselines(layer, inp, w, res, timed)
     # selection variants on the layer's scores: an 8-budget sweep in one launch vs
     # eight single-budget launches, and random-K from caller-drawn keys
     n_doc = np.asarray(inp.doc_end) - np.asarray(inp.doc_begin)
@@ -701,6 +762,7 @@ def run_extras(args):
         "extras": args.workload, "tokens": w.total_tokens, "kept": w.kept_lengths(),
         "stage_us": {s: round(v, 2) for s, v in stage_us.items()},
         "gated_layer_us": round(gated_total, 2),
+        "library_same_shapes_us": library,
         "bias_overhead": {"with_bias_us": round(with_bias, 2), "no_bias_us": round(no_bias, 2),
                           "ratio": round(with_bias / no_bias, 4)},
         "ungated_attention": {"us": round(ungated, 2), "tflops": round(full_flops / ungated / 1e6, 1),
