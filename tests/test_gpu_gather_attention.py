@@ -63,6 +63,15 @@ def test_gather_varlen_small_and_empty(oracle):
     _gather_case(oracle, w, seed=5)
 
 
+@pytest.mark.parametrize("dtype,d_model", [("bf16", 32768), ("fp32", 16384)])
+def test_gather_rows_wider_than_a_stage(oracle, dtype, d_model):
+    # a kept row of more than 48 KB over its four tensors does not fit one stage of
+    # the bulk-copy ring: the warp-per-(row, tensor) kernel moves it
+    w = gen.Workload("wide", (300, 0, 77), (20, 0, 5), (40, 1, 100), d_model, 32, 4, 2, 64, dtype,
+                     1, 13)
+    _gather_case(oracle, w, seed=3)
+
+
 # ---- attention -----------------------------------------------------------------
 
 def _attn_case(oracle, lens, Hq, Hkv, dh, dtype, algo, bias=True, seed=0, rows=None,
