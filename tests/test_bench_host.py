@@ -123,3 +123,32 @@ def test_committed_traffic_records_name_existing_sources(bench):
                                                rec["source"])), (kernel, wl)
             assert rec["bytes_per_launch"] == rec["read"] + rec["write"], (kernel, wl)
             assert len(rec["sha256"]) == 16
+
+
+def _run_bench(args, env_extra=None, timeout=300):
+    import subprocess
+    import sys
+    env = dict(os.environ, **(env_extra or {}))
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=timeout)
+    assert p.returncode == 0, p.stderr[-2000:]
+    return [json.loads(x) for x in p.stdout.splitlines() if x.startswith("{")]
+
+
+def test_reference_arm_prints_one_contract_line():
+    # the oracle on the host cores: one bounded sample per step, no device
+    (line,) = _run_bench(["--impl", "reference", "--workload", "tiny_fp32", "--steps", "1",
+                          "--warmup", "0"])
+    assert line["impl"] == "reference" and line["metric"] == "gated-prefill input tok/s"
+    assert line["unit"] == "tok/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["dtype"] == "f64" and line["vs_baseline"] is None
+    assert line["config"]["workload"] == "tiny_fp32"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tok/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    assert _run_bench(["--impl", "reference", "--workload", "tiny_fp32", "--steps", "1",
+                       "--warmup", "0"], env_extra={"RANK": "1", "WORLD_SIZE": "2"}) == []
